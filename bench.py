@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of one DELTA decode step (every layer of the stack) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+
+Default workload: the Qwen-7B-shaped stack in bf16 (28 layers: 0-1 full, delta-layers 2
+and 14, 24 sparse; 28 query / 4 KV heads, head_dim 128; batch 1, context 8192, 16-token
+pages; budget 1024 tokens + 16-token sink + 256-token recency window), synthetic inputs with
+32 planted salient keys per (layer, KV head).  A step is one decode step: kv_append, then
+full, delta or sparse attention, for each of the 28 layers, captured as one CUDA graph.
+
+Timing: W untimed replays, then K timed replays, L2 flushed (a 2x L2-sized write) before every
+replay outside the events; CUDA events on the replay stream; max over ranks.  Prints one JSON
+line.  With --gpus N > 1 (torchrun) every rank runs an independent replica (the path does
+not shard across GPUs) and the reported time is the slowest rank's.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "us_per_decode_step_layer_stack"
+UNIT = "us/step"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        mhz, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        return dist, int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
+    return None, 0, 1, 0
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    import torch
+    if dist is not None:
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+# ---------------------------------------------------------------------------- accounting
+def attended_tokens(cfg, case):
+    """(delta_stack_tokens, full_stack_tokens) attended per step, summed over layers and sequences.
+
+    Sparse layers attend the tokens of the selected pages: every sink/recency page plus k
+    candidate pages, the last page partial (computed from the selection rule's page counts).
+    """
+    P = cfg.page_size
+    kinds = cfg.layer_kinds()
+    full_tok = 0
+    sparse_tok = 0
+    for n in case.n.tolist():
+        N = -(-n // P)
+        sinkP = -(-min(cfg.sink_tokens, n) // P)
+        recStart = max(n - cfg.recency_tokens, 0) // P if cfg.recency_tokens > 0 else N
+        forced = set(range(sinkP)) | set(range(recStart, N))
+        cand = N - len(forced)
+        pages = len(forced) + min(cfg.budget_pages, cand)
+        tail_missing = (N * P - n) if (N - 1) in forced or cand <= cfg.budget_pages else 0
+        sparse_tok += pages * P - tail_missing
+        full_tok += n
+    n_sparse = kinds.count("sparse")
+    n_dense = len(kinds) - n_sparse
+    return n_dense * full_tok + n_sparse * sparse_tok, len(kinds) * full_tok, full_tok, sparse_tok
+
+
+# ---------------------------------------------------------------------------- reference arm
+class OracleSample:
+    """The fp64 oracle on one full, one delta and one sparse layer of sequence 0 (inputs
+    generated once, outside any timing); a step estimate scales them to the whole stack."""
+
+    def __init__(self, cfg, case):
+        import numpy as np
+        from oracle import delta_oracle as O
+        from synth import rng
+        self.cfg, self.O = cfg, O
+        kinds = cfg.layer_kinds()
+        self.kinds = kinds
+        self.l_delta = kinds.index("delta")
+        self.l_full = kinds.index("full") if "full" in kinds else self.l_delta
+        self.l_sparse = kinds.index("sparse")
+        b = 0
+        self.n = int(case.n[b])
+
+        def kv(l):
+            K = np.stack([case.kv_logical(rng.T_K, l, b, g) for g in range(cfg.num_kv_heads)]).astype(np.float64)
+            V = np.stack([case.kv_logical(rng.T_V, l, b, g) for g in range(cfg.num_kv_heads)]).astype(np.float64)
+            return K, V
+
+        self.data = {l: (case.q(l)[b].astype(np.float64),) + kv(l) for l in (self.l_full, self.l_delta, self.l_sparse)}
+        self.sel = self._select(self.data[self.l_delta])
+
+    def _select(self, qkv):
+        c, O = self.cfg, self.O
+        _, p = O.full_attention(*qkv)
+        return O.select_pages(O.page_scores(p, c.page_size), self.n, c.page_size, c.budget_pages, c.sink_tokens,
+                              c.recency_tokens)
+
+    def layer_us(self, min_seconds: float = 0.0, max_reps: int = 200) -> dict:
+        """Wall-clock microseconds per layer of each kind for one sequence."""
+        O, c = self.O, self.cfg
+        fns = {"full": lambda: O.full_attention(*self.data[self.l_full]),
+               "delta": lambda: self._select(self.data[self.l_delta]),
+               "sparse": lambda: O.sparse_attention(*self.data[self.l_sparse], self.sel, c.page_size)}
+        out = {}
+        for name, fn in fns.items():
+            k, t0 = 0, time.perf_counter()
+            while True:
+                fn()
+                k += 1
+                el = time.perf_counter() - t0
+                if el >= min_seconds / 3 or k >= max_reps:
+                    break
+            out[name] = el / k * 1e6
+        return out
+
+    def step_us(self, times: dict) -> tuple:
+        """(delta-stack us per step, full-stack us per step) for the whole batch."""
+        n_kind = {k: self.kinds.count(k) for k in ("full", "delta", "sparse")}
+        delta_us = self.cfg.batch * sum(n_kind[k] * times[k] for k in times)
+        full_us = self.cfg.batch * len(self.kinds) * times["full"]
+        return delta_us, full_us
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    dist, rank, world, local = dist_init()
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    from synth import configs as C
+    from synth.case import Case
+    cfg = C.CONFIGS[args.config]
+    case = Case(cfg)
+    sample = OracleSample(cfg, case)
+    per_step = []
+    desc = None
+    for i in range(args.warmup + args.steps):
+        times = sample.layer_us(max_reps=1)
+        d_us, _ = sample.step_us(times)
+        if i >= args.warmup:
+            per_step.append(d_us)
+        desc = times
+    value = statistics.mean(per_step)
+    cores = blas_threads()
+    sample = (f"fp64 numpy oracle, sequence 0, one full / delta / sparse layer per step "
+              f"({', '.join(f'{k} {v:.0f} us' for k, v in desc.items())}), scaled to {cfg.num_layers} layers "
+              f"x batch {cfg.batch}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1000, 6),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "context": int(case.n.max()), "layers": cfg.num_layers},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    from long_context_layer_b200 import _native as NAT
+    from long_context_layer_b200.stack import DeltaStack
+    from synth import configs as C
+    from synth.case import Case
+    from synth.gpu import DeviceCase
+
+    dist, rank, world, local = dist_init()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = C.CONFIGS[args.config]
+    case = Case(cfg)
+    dc = DeviceCase(case, device=device, prefill="append")
+    kinds = cfg.layer_kinds()
+    mk = lambda kk: DeltaStack(kk, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr, dc.indices,
+                               dc.kv_len, case.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages,
+                               cfg.sink_tokens, cfg.recency_tokens)
+    delta_stack = mk(kinds)
+    full_stack = mk(["full"] * cfg.num_layers)
+    args_step = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    g_delta = delta_stack.capture(*args_step)
+    g_full = full_stack.capture(*args_step)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(replay, k, warm):
+        for _ in range(warm):
+            flush.fill_(1)
+            replay()
+        barrier(dist, device)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        for s, e in ev:
+            flush.fill_(1)
+            s.record(stream)
+            replay()
+            e.record(stream)
+        barrier(dist, device)
+        return [s.elapsed_time(e) * 1000.0 for s, e in ev]   # us
+
+    sampler = ClockSampler(device.index if not os.environ.get("CUDA_VISIBLE_DEVICES") else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[device.index]))
+    sampler.start()
+    time.sleep(0.3)
+    t_delta = timed(g_delta.replay, args.steps, args.warmup)
+    clocks = sampler.stop()
+    t_full = timed(g_full.replay, max(args.steps // 2, 3), 3)
+    us_delta = max_over_ranks(dist, statistics.mean(t_delta), device)
+    us_full = max_over_ranks(dist, statistics.mean(t_full), device)
+
+    # -- dominant kernel: the decode kernel of a full layer, timed alone (one launch per call)
+    st = stream.cuda_stream
+    d0 = delta_stack
+    layer0 = 0
+
+    def full_call():
+        NAT.full_attn(d0.desc, d0.pt, dc.q[layer0], dc.k_pools[layer0], dc.v_pools[layer0], dc.out[layer0],
+                      d0.workspace, d0.ws_bytes, st)
+
+    t_kernel = timed(full_call, max(args.steps, 20), 3)
+    us_kernel = max_over_ranks(dist, statistics.mean(t_kernel), device)
+    e = 2 if cfg.dtype == "bf16" else 4
+    kv_bytes = int(case.n.sum()) * 2 * cfg.num_kv_heads * cfg.head_dim * e
+    qo_bytes = 2 * cfg.batch * cfg.num_q_heads * cfg.head_dim * e
+    alg_bytes = kv_bytes + qo_bytes
+    peak, peak_kind = load_peaks()
+    achieved = alg_bytes / (us_kernel * 1e-6) / 1e9
+
+    # -- end to end through the public API: pinned host inputs in, outputs out, every step
+    q_h = dc.q.cpu().pin_memory()
+    kn_h, vn_h = dc.k_new.cpu().pin_memory(), dc.v_new.cpu().pin_memory()
+    out_h = torch.empty_like(dc.out, device="cpu").pin_memory()
+    sel_h = torch.empty_like(delta_stack.sel_pages, device="cpu").pin_memory()
+
+    def e2e_step():
+        dc.q.copy_(q_h, non_blocking=True)
+        dc.k_new.copy_(kn_h, non_blocking=True)
+        dc.v_new.copy_(vn_h, non_blocking=True)
+        g_delta.replay()
+        out_h.copy_(dc.out, non_blocking=True)
+        sel_h.copy_(delta_stack.sel_pages, non_blocking=True)
+
+    t_e2e = timed(e2e_step, args.steps, 3)
+    us_e2e = max_over_ranks(dist, statistics.mean(t_e2e), device)
+    h2d = (q_h.numel() + kn_h.numel() + vn_h.numel()) * e
+    d2h = out_h.numel() * e + sel_h.numel() * 4
+
+    tok_delta, tok_full, _, _ = attended_tokens(cfg, case)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(cfg, case)
+        times = sample.layer_us(min_seconds=args.cpu_seconds)
+        d_us, f_us = sample.step_us(times)
+        cpu = {"value": round(d_us, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": ("fp64 numpy oracle on the host cores, sequence 0, one full / delta / sparse layer "
+                          f"repeated for ~{args.cpu_seconds:.0f} s ({', '.join(f'{k} {v:.0f} us' for k, v in times.items())}), "
+                          f"scaled to the {cfg.num_layers}-layer step x batch {cfg.batch}"),
+               "full_stack_value": round(f_us, 1)}
+    launches = delta_stack.launches_per_step() * args.steps
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(us_delta, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(us_delta / 1000, 6), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "layers": cfg.num_layers, "delta_layers": list(cfg.delta_layers),
+                       "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
+                       "batch": cfg.batch, "context": int(case.n.max()), "page_size": cfg.page_size,
+                       "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
+                       "recency_tokens": cfg.recency_tokens, "l2": "flushed before every timed replay",
+                       "parallelism": f"replicas x{world}"},
+            "full_stack_us": round(us_full, 3),
+            "speedup_vs_full_stack": round(us_full / us_delta, 3),
+            "attended_token_reduction": round(tok_full / tok_delta, 3),
+            "roofline": {"kernel": "decode_kernel (full layer, fused split merge)", "bound": "hbm",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                         "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_kernel, 3),
+                         "traffic": None},
+            "e2e": {"value": round(us_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    # release graphs before tearing down the process group
+    del g_delta, g_full
+    delta_stack.graph = None
+    full_stack.graph = None
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

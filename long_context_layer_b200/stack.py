@@ -1,0 +1,110 @@
+"""One DELTA decode step over a whole layer stack, through the C ABI.
+
+Layer schedule (DELTA: Dynamic Layer-Aware Token Attention, ai.info summary,
+"Methodology in Plain English"): layers before the first delta-layer run full
+attention; a delta-layer runs full attention and refreshes the page selection;
+every other layer runs sparse attention over the selection of the most recent
+delta-layer of the same decode step.  Every layer first appends the current
+token's k and v to its own paged pool (the cache is kept in full).
+
+The runner only sequences C-ABI calls on one CUDA stream; it can capture the
+whole step in a CUDA graph so one replay launches every kernel of the step.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _native as N
+
+FULL, DELTA, SPARSE = "full", "delta", "sparse"
+
+
+def layer_kinds(num_layers: int, delta_layers) -> list:
+    first = min(delta_layers)
+    return [DELTA if l in delta_layers else (FULL if l < first else SPARSE) for l in range(num_layers)]
+
+
+class DeltaStack:
+    """Buffers and call sequence of one decode step.
+
+    Tensors (all on one CUDA device):
+      indptr [B+1], indices [nnz], kv_len [B]  int32 page table shared by all layers
+      k_pools[l], v_pools[l]                   [num_phys_pages, Hkv, 16, D] per layer
+      q [L, B, Hq, D], k_new / v_new [L, B, Hkv, D], out [L, B, Hq, D]
+    """
+
+    def __init__(self, kinds, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: torch.dtype,
+                 indptr: torch.Tensor, indices: torch.Tensor, kv_len: torch.Tensor, max_pages_per_seq: int,
+                 num_phys_pages: int, budget_pages: int = 0, sink_tokens: int = 0, recency_tokens: int = 0,
+                 sm_scale: float = 0.0, keep_scores: bool = False):
+        self.kinds = list(kinds)
+        self.device = indptr.device
+        self.batch = int(kv_len.numel())
+        self.dtype = dtype
+        dt = N.DELTA_BF16 if dtype == torch.bfloat16 else N.DELTA_F32
+        if dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("dtype must be bfloat16 or float32")
+        self.desc = N.DeltaDesc(num_q_heads, num_kv_heads, head_dim, 16, dt, sm_scale, num_phys_pages)
+        self.indptr, self.indices, self.kv_len = indptr, indices, kv_len
+        self.pt = N.DeltaPageTable(indptr.data_ptr(), indices.data_ptr(), kv_len.data_ptr(), self.batch,
+                                   max_pages_per_seq)
+        self.sp = N.DeltaSelectParams(budget_pages, sink_tokens, recency_tokens, N.DELTA_HEAD_SUM)
+        self.max_pages = max_pages_per_seq
+        self.ws_bytes = N.workspace_size(self.desc, self.batch, max_pages_per_seq)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        N.workspace_init(self.workspace, self.ws_bytes, torch.cuda.current_stream(self.device).cuda_stream)
+        self.sel_stride = max(N.sel_capacity(self.sp), 1)
+        self.delta_layers = [l for l, k in enumerate(self.kinds) if k == DELTA]
+        nd = max(len(self.delta_layers), 1)
+        self.sel_cnt = torch.zeros(nd, self.batch, dtype=torch.int32, device=self.device)
+        self.sel_pages = torch.zeros(nd, self.batch, self.sel_stride, dtype=torch.int32, device=self.device)
+        self.page_scores = (torch.zeros(nd, self.batch, max_pages_per_seq, dtype=torch.float32, device=self.device)
+                            if keep_scores else None)
+        if any(k == SPARSE for k in self.kinds):
+            first_sparse = self.kinds.index(SPARSE)
+            if not any(k == DELTA for k in self.kinds[:first_sparse]):
+                raise ValueError("a sparse layer needs an earlier delta-layer")
+        self.graph = None
+
+    # ------------------------------------------------------------------ one step
+    def launches_per_step(self, append: bool = True) -> int:
+        per = {FULL: 1, DELTA: 2, SPARSE: 1}
+        return sum(per[k] + (1 if append else 0) for k in self.kinds)
+
+    def step(self, q, k_new, v_new, k_pools, v_pools, out, append: bool = True, stream: int | None = None):
+        st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
+        d, pt, ws, wb = self.desc, self.pt, self.workspace, self.ws_bytes
+        cur = -1
+        for l, kind in enumerate(self.kinds):
+            if append:
+                N.kv_append(d, pt, k_new[l], v_new[l], k_pools[l], v_pools[l], st)
+            if kind == FULL:
+                N.full_attn(d, pt, q[l], k_pools[l], v_pools[l], out[l], ws, wb, st)
+            elif kind == DELTA:
+                cur = self.delta_layers.index(l)
+                scores = self.page_scores[cur] if self.page_scores is not None else None
+                N.select_attn(d, pt, self.sp, q[l], k_pools[l], v_pools[l], out[l], self.sel_cnt[cur],
+                              self.sel_pages[cur], self.sel_stride, scores, ws, wb, st)
+            else:
+                N.sparse_attn(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l], k_pools[l],
+                              v_pools[l], out[l], ws, wb, st)
+
+    # ------------------------------------------------------------------ CUDA graph
+    def capture(self, *args, **kw) -> torch.cuda.CUDAGraph:
+        """Capture one step (same arguments as step) into a CUDA graph and return it."""
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self.step(*args, **kw)          # warm: sets per-device kernel attributes outside capture
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step(*args, **kw)
+        self.graph = g
+        return g
+
+    def selection(self, delta_index: int = -1) -> list:
+        """Host copy of a delta-layer's selection: list (per sequence) of ascending logical pages."""
+        cnt = self.sel_cnt[delta_index].cpu().tolist()
+        pages = self.sel_pages[delta_index].cpu()
+        return [pages[b, :cnt[b]].tolist() for b in range(self.batch)]

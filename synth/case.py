@@ -86,13 +86,17 @@ class Case:
             hi = int(self.n[b]) - 1 - c.recency_tokens - c.drift_shift * ((c.steps - 1) // c.drift_every)
         else:
             hi = int(self.n[b]) - c.recency_tokens
-        if hi - lo < c.planted:
-            hi = lo + c.planted
+        hi = min(hi, int(self.n[b]) - 1)          # the current token is never planted
+        count = min(c.planted, max(hi - lo, 0))   # short contexts plant fewer keys
+        if count == 0:
+            out = np.zeros(0, dtype=np.int64)
+            self._plant_cache[ck] = out
+            return out
         if layer == 0:
             prev = None
         else:
             prev = self._base_positions(layer - 1, b, g)
-        keep = int(round(c.planted_overlap * c.planted)) if prev is not None else 0
+        keep = min(int(round(c.planted_overlap * count)), len(prev)) if prev is not None else 0
         uid = (layer * 64 + b) * 64 + g
         chosen = []
         if keep:
@@ -100,7 +104,7 @@ class Case:
             chosen = [int(prev[i]) for i in order[:keep]]
         taken = set(chosen)
         draw = 0
-        while len(chosen) < c.planted:
+        while len(chosen) < count:
             p = int(rng.randint(self.key, rng.aux_counter(rng.SALT_PLANT_DRAW + uid, [draw]), lo, hi)[0])
             draw += 1
             if p not in taken:

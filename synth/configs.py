@@ -39,6 +39,7 @@ class StackConfig:
     recency_tokens: int
     context: int = 0                # fixed n_b (tokens attended, current token included); 0 -> drawn
     context_range: tuple = ()       # (lo, hi) inclusive range for per-sequence draws
+    context_list: tuple = ()        # explicit n_b per sequence (overrides the two above)
     planted: int = 0                # salient keys per (layer, b, kv head)
     planted_overlap: float = 0.8
     pool_pages_per_layer: int = 0   # 0 -> exactly the pages the sequences need
@@ -70,7 +71,9 @@ class StackConfig:
 
     def contexts(self, step: int = 0) -> list:
         """n_b for every sequence at a decode step (the appended token included)."""
-        if self.context:
+        if self.context_list:
+            base = list(self.context_list)
+        elif self.context:
             base = [self.context] * self.batch
         else:
             lo, hi = self.context_range
@@ -79,7 +82,7 @@ class StackConfig:
         return [n + step for n in base]
 
     def max_context(self) -> int:
-        top = self.context if self.context else self.context_range[1]
+        top = max(self.context_list) if self.context_list else (self.context if self.context else self.context_range[1])
         return top + self.steps - 1
 
     def with_(self, **kw) -> "StackConfig":

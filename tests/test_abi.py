@@ -1,0 +1,118 @@
+"""The C-ABI library loads, exports every symbol the header declares, and rejects bad
+arguments on the host before launching anything (no GPU needed for these paths)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "delta_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_layer_b200 import build
+    build.build()
+    import long_context_layer_b200 as lib
+    return lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:size_t|delta_status|int32_t|const char\*)\s+(delta_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_four_calls():
+    fns = declared_functions()
+    for name in ("delta_kv_append", "delta_full_attn", "delta_select_attn", "delta_sparse_attn"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", L._native.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    assert sorted(L._native.EXPORTED) == declared_functions()
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.status_string(s) and L.status_string(s) != "unknown status"
+    assert L.status_string(99) == "unknown status"
+
+
+def _desc(L, **kw):
+    d = dict(num_q_heads=28, num_kv_heads=4, head_dim=128, page_size=16, dtype=L.DELTA_BF16, sm_scale=0.0,
+             num_phys_pages=512)
+    d.update(kw)
+    return L.DeltaDesc(**d)
+
+
+FAKE = 1 << 40  # never dereferenced: every call below fails validation first
+
+
+def _pt(L, batch=1, maxp=512):
+    return L.DeltaPageTable(FAKE, FAKE, FAKE, batch, maxp)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_q_heads=27), 1),          # not a multiple of the KV heads
+    (dict(head_dim=96), 2),             # unsupported head dim
+    (dict(page_size=32), 2),            # unsupported page size
+    (dict(num_q_heads=36), 2),          # group of 9 > 8
+    (dict(dtype=7), 1),
+    (dict(sm_scale=-1.0), 1),
+])
+def test_bad_descriptor_rejected(L, kw, status):
+    s = L.full_attn(_desc(L, **kw), _pt(L), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, 0, check=False)
+    assert s == status
+
+
+def test_null_pointers_and_workspace_rejected(L):
+    d = _desc(L)
+    assert L.full_attn(d, _pt(L), None, FAKE, FAKE, FAKE, FAKE, 1 << 30, 0, check=False) == 1
+    assert L.full_attn(d, L.DeltaPageTable(None, FAKE, FAKE, 1, 512), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, 0,
+                       check=False) == 1
+    assert L.full_attn(d, _pt(L), FAKE, FAKE, FAKE, FAKE, None, 1 << 30, 0, check=False) == 3
+    assert L.full_attn(d, _pt(L), FAKE, FAKE, FAKE, FAKE, FAKE + 8, 1 << 30, 0, check=False) == 3   # misaligned
+    need = L.workspace_size(d, 1, 512)
+    assert need > 0
+    assert L.full_attn(d, _pt(L), FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, 0, check=False) == 3
+    assert L.full_attn(d, _pt(L), FAKE + 4, FAKE, FAKE, FAKE, FAKE, need, 0, check=False) == 1     # misaligned q
+
+
+def test_select_arguments_rejected(L):
+    d = _desc(L)
+    sp = L.DeltaSelectParams(64, 16, 256, L.DELTA_HEAD_SUM)
+    cap = L.sel_capacity(sp)
+    assert cap == 64 + 1 + 17
+    ws = L.workspace_size(d, 1, 512)
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert L.select_attn(d, _pt(L), sp, *args[:4], FAKE, FAKE, cap - 1, None, FAKE, ws, 0, check=False) == 1
+    sp_max = L.DeltaSelectParams(64, 16, 256, L.DELTA_HEAD_MAX)
+    assert L.select_attn(d, _pt(L), sp_max, *args[:4], FAKE, FAKE, cap, None, FAKE, ws, 0, check=False) == 2
+    sp_bad = L.DeltaSelectParams(-1, 16, 256, L.DELTA_HEAD_SUM)
+    assert L.select_attn(d, _pt(L), sp_bad, *args[:4], FAKE, FAKE, cap, None, FAKE, ws, 0, check=False) == 1
+    assert L.select_attn(d, _pt(L, maxp=40000), sp, *args[:4], FAKE, FAKE, cap, None, FAKE,
+                         L.workspace_size(d, 1, 40000), 0, check=False) == 2
+    assert L.select_attn(d, _pt(L), sp, *args[:4], None, FAKE, cap, None, FAKE, ws, 0, check=False) == 1
+
+
+def test_sparse_and_append_arguments_rejected(L):
+    d = _desc(L)
+    ws = L.workspace_size(d, 1, 512)
+    assert L.sparse_attn(d, _pt(L), None, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 0, check=False) == 1
+    assert L.sparse_attn(d, _pt(L), FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 0, check=False) == 1
+    assert L.kv_append(d, _pt(L), None, FAKE, FAKE, FAKE, 0, check=False) == 1
+    assert L.kv_append(_desc(L, head_dim=80), _pt(L), FAKE, FAKE, FAKE, FAKE, 0, check=False) == 2
+
+
+def test_empty_batch_is_a_no_op(L):
+    d = _desc(L)
+    pt = L.DeltaPageTable(None, None, None, 0, 0)
+    assert L.full_attn(d, pt, None, None, None, None, None, 0, 0, check=False) == 0
+    assert L.kv_append(d, pt, None, None, None, None, 0, check=False) == 0
