@@ -35,7 +35,9 @@ def nvcc() -> str:
 def build(force: bool = False, verbose: bool = False) -> list:
     built = []
     for src, out, extra in TARGETS:
-        deps = [src] + [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
+        csrc = os.path.dirname(src)
+        deps = [os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h"))]
+        deps += [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
         if not force and os.path.exists(out) and os.path.getmtime(out) >= max(os.path.getmtime(d) for d in deps):
             continue
         cmd = [nvcc()] + ARCH + COMMON + extra + [src, "-o", out]

@@ -50,7 +50,8 @@ class DeviceCase:
     writes every attended token (for tests that skip the append).
     """
 
-    def __init__(self, case: Case, device="cuda", layers=None, prefill="append", pool_pages: int | None = None):
+    def __init__(self, case: Case, device="cuda", layers=None, prefill="append", pool_pages: int | None = None,
+                 garbage: float | None = None):
         self.case = case
         cfg = case.cfg
         self.cfg = cfg
@@ -68,6 +69,9 @@ class DeviceCase:
         for l in self.layers:
             kp = torch.empty((self.num_phys_pages, Hkv, 16, D), dtype=self.dtype, device=self.device)
             vp = torch.empty_like(kp)
+            if garbage is not None:           # what unwritten cache slots hold (e.g. NaN)
+                kp.fill_(garbage)
+                vp.fill_(garbage)
             self._fill(kp, rng.T_K, l)
             self._fill(vp, rng.T_V, l)
             self._plant(kp, l)

@@ -111,6 +111,23 @@ def test_full_attn_matches_oracle(L, G, Hkv, D, dtype, ctx):
         assert_close(out[b], ref, dtype, f"b={b} n={n}")
 
 
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("bf16", 128), ("bf16", 64)])
+def test_unwritten_slots_holding_nan_do_not_leak(L, dtype, D):
+    # the last page of each sequence is partial; its unwritten slots hold NaN
+    from synth.gpu import DeviceCase
+    cfg = make_cfg(7, 2, D, dtype, [33, 1000, 17])
+    case = Case(cfg)
+    dc = DeviceCase(case, prefill="all", garbage=float("nan"))
+    desc, pt = make_desc(L, cfg, dc), make_pt(L, dc)
+    ws, nb = workspace(L, desc, dc)
+    L.full_attn(desc, pt, dc.q[0], dc.k_pools[0], dc.v_pools[0], dc.out[0], ws, nb, stream())
+    out = dc.out[0].float().cpu().numpy()
+    assert np.isfinite(out).all()
+    for b in range(3):
+        K, V = oracle_kv(case, 0, b)
+        assert_close(out[b], O.full_attention(case.q(0)[b].astype(np.float64), K, V)[0], dtype, f"b={b}")
+
+
 def test_empty_sequence_gives_zero_output(L):
     cfg = make_cfg(4, 1, 64, "f32", [0, 20])
     cfg = cfg.with_(context_list=(0, 20))
@@ -225,10 +242,11 @@ def test_kv_append_writes_exactly_one_slot(L, dtype, D):
     cfg = make_cfg(4, 2, D, dtype, [33, 16, 1, 100], extra_pool=5)
     dc = device_case(cfg, prefill="append")
     desc, pt = make_desc(L, cfg, dc), make_pt(L, dc)
-    before_k, before_v = dc.k_pools[0].clone(), dc.v_pools[0].clone()
+    bits = torch.int16 if dtype == "bf16" else torch.int32           # compare bytes: garbage may hold NaNs
+    before_k, before_v = dc.k_pools[0].view(bits).clone(), dc.v_pools[0].view(bits).clone()
     L.kv_append(desc, pt, dc.k_new[0], dc.v_new[0], dc.k_pools[0], dc.v_pools[0], stream())
     torch.cuda.synchronize()
-    changed = (dc.k_pools[0] != before_k).any(-1) | (dc.v_pools[0] != before_v).any(-1)
+    changed = (dc.k_pools[0].view(bits) != before_k).any(-1) | (dc.v_pools[0].view(bits) != before_v).any(-1)
     for b, n in enumerate(cfg.context_list):
         for g in range(2):
             for t, new in ((rng.T_K, dc.k_new[0]), (rng.T_V, dc.v_new[0])):
