@@ -288,16 +288,23 @@ def run_ours(args):
     g_full = full_stack.capture(*args_step)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+    flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
+
+    def flush_l2():
+        # write a buffer twice the size of L2, then read another one, so no dirty lines of the
+        # flush are left to be written back inside the timed region
+        flush.fill_(1)
+        flush_rd.sum()
 
     def timed(replay, k, warm):
         for _ in range(warm):
-            flush.fill_(1)
+            flush_l2()
             replay()
         barrier(dist, device)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         for s, e in ev:
-            flush.fill_(1)
+            flush_l2()
             s.record(stream)
             replay()
             e.record(stream)
@@ -325,6 +332,27 @@ def run_ours(args):
 
     t_kernel = timed(full_call, max(args.steps, 20), 3)
     us_kernel = max_over_ranks(dist, statistics.mean(t_kernel), device)
+
+    # -- per-call breakdown (each call timed alone, L2 flushed before it)
+    lk = kinds.index("delta")
+    ls = kinds.index("sparse")
+    di = d0.delta_layers.index(lk)
+
+    def append_call():
+        NAT.kv_append(d0.desc, d0.pt, dc.k_new[0], dc.v_new[0], dc.k_pools[0], dc.v_pools[0], st)
+
+    def select_call():
+        NAT.select_attn(d0.desc, d0.pt, d0.sp, dc.q[lk], dc.k_pools[lk], dc.v_pools[lk], dc.out[lk], d0.sel_cnt[di],
+                        d0.sel_pages[di], d0.sel_stride, None, d0.workspace, d0.ws_bytes, st)
+
+    def sparse_call():
+        NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[ls], dc.k_pools[ls],
+                        dc.v_pools[ls], dc.out[ls], d0.workspace, d0.ws_bytes, st)
+
+    n_b = max(args.steps // 2, 10)
+    breakdown = {name: round(max_over_ranks(dist, statistics.mean(timed(fn, n_b, 3)), device), 3)
+                 for name, fn in (("kv_append", append_call), ("full_attn", full_call),
+                                  ("select_attn", select_call), ("sparse_attn", sparse_call))}
     e = 2 if cfg.dtype == "bf16" else 4
     kv_bytes = int(case.n.sum()) * 2 * cfg.num_kv_heads * cfg.head_dim * e
     qo_bytes = 2 * cfg.batch * cfg.num_q_heads * cfg.head_dim * e
@@ -372,7 +400,7 @@ def run_ours(args):
                        "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
                        "batch": cfg.batch, "context": int(case.n.max()), "page_size": cfg.page_size,
                        "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
-                       "recency_tokens": cfg.recency_tokens, "l2": "flushed before every timed replay",
+                       "recency_tokens": cfg.recency_tokens, "l2": "flushed before every timed replay (2xL2 write, then 2xL2 read)",
                        "parallelism": f"replicas x{world}"},
             "full_stack_us": round(us_full, 3),
             "speedup_vs_full_stack": round(us_full / us_delta, 3),
@@ -382,6 +410,7 @@ def run_ours(args):
                          "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                          "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_kernel, 3),
                          "traffic": None},
+            "breakdown_us_per_call": breakdown,
             "e2e": {"value": round(us_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks,

@@ -10,6 +10,7 @@
  * exposes one call per step of that decode path:
  *
  *   delta_kv_append    write the current token's k, v into the paged cache
+ *                      (delta_kv_append_layers: every layer of a step in one launch)
  *   delta_full_attn    full decode attention (initial layers)
  *   delta_select_attn  full decode attention + per-page scores + page selection (delta-layers)
  *   delta_sparse_attn  decode attention over the selected pages only (sparse layers)
@@ -36,6 +37,11 @@
  *     sel_pages       [batch][sel_stride] ascending LOGICAL page ids, sel_cnt[batch] valid
  *     page_scores     [batch][max_pages_per_seq] fp32
  * - Grouped-query attention: query head h reads KV head h / (num_q_heads/num_kv_heads).
+ * - Kernels are launched with programmatic dependent launch: a kernel may be scheduled while
+ *   the previous kernel of the stream drains, and waits for it before reading q, the pools or a
+ *   selection.  The page table and kv_len are treated as inputs of the whole decode step and may
+ *   be read before that wait, so a kernel that writes them must complete before the call
+ *   (any kernel launched without programmatic dependent launch does).
  * - Host-detectable errors return a status and launch nothing.  A launch failure
  *   returns DELTA_ERR_CUDA.  Device-detected errors (a page id outside the pool, a
  *   kv_len beyond the sequence's pages, a selection entry outside the context, a
@@ -121,6 +127,14 @@ int32_t delta_sel_capacity(const delta_select_params* sp, int32_t page_size);
 delta_status delta_kv_append(const delta_desc* desc, const delta_page_table* pt,
                              const void* k_new, const void* v_new,
                              void* k_pool, void* v_pool, void* stream);
+
+/* The same append for every layer of a decode step in one launch: layer l copies k_new[l],
+ * v_new[l] into k_pools[l], v_pools[l].  The four arguments are HOST arrays of num_layers
+ * device pointers (num_layers <= 64; more gives DELTA_ERR_UNSUPPORTED); all layers share the
+ * descriptor and the page table. */
+delta_status delta_kv_append_layers(const delta_desc* desc, const delta_page_table* pt, int32_t num_layers,
+                                    const void* const* k_new, const void* const* v_new,
+                                    void* const* k_pools, void* const* v_pools, void* stream);
 
 /* Full decode attention: o[b][h] = sum_t softmax_t(sm_scale * q[b][h].k_t) v_t over the
  * kv_len[b] cached tokens of KV head h/G (initial layers "run ordinary full attention",

@@ -25,6 +25,7 @@ DELTA_HEAD_SUM, DELTA_HEAD_MAX = 0, 1
 
 EXPORTED = [
     "delta_workspace_size", "delta_workspace_init", "delta_sel_capacity", "delta_kv_append",
+    "delta_kv_append_layers",
     "delta_full_attn", "delta_select_attn", "delta_sparse_attn", "delta_read_device_error",
     "delta_status_string",
 ]
@@ -59,6 +60,9 @@ lib.delta_sel_capacity.argtypes = [_SP, _i32]
 lib.delta_sel_capacity.restype = _i32
 lib.delta_kv_append.argtypes = [_D, _PT, _vp, _vp, _vp, _vp, _vp]
 lib.delta_kv_append.restype = _i32
+_vpp = ctypes.POINTER(ctypes.c_void_p)
+lib.delta_kv_append_layers.argtypes = [_D, _PT, _i32, _vpp, _vpp, _vpp, _vpp, _vp]
+lib.delta_kv_append_layers.restype = _i32
 lib.delta_full_attn.argtypes = [_D, _PT, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.delta_full_attn.restype = _i32
 lib.delta_select_attn.argtypes = [_D, _PT, _SP, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]
@@ -112,6 +116,19 @@ def kv_append(desc, pt, k_new, v_new, k_pool, v_pool, stream: int = 0, check: bo
     s = lib.delta_kv_append(ctypes.byref(desc), ctypes.byref(pt), ptr(k_new), ptr(v_new), ptr(k_pool),
                             ptr(v_pool), stream)
     return _check(s, "delta_kv_append") if check else s
+
+
+def _ptr_array(xs):
+    return (ctypes.c_void_p * len(xs))(*[ptr(x) for x in xs])
+
+
+def kv_append_layers(desc, pt, k_new, v_new, k_pools, v_pools, stream: int = 0, check: bool = True) -> int:
+    """k_new, v_new, k_pools, v_pools: sequences (one entry per layer) of device tensors or pointers."""
+    n = len(k_pools)
+    s = lib.delta_kv_append_layers(ctypes.byref(desc), ctypes.byref(pt), n, _ptr_array([k_new[l] for l in range(n)]),
+                                   _ptr_array([v_new[l] for l in range(n)]), _ptr_array(list(k_pools)),
+                                   _ptr_array(list(v_pools)), stream)
+    return _check(s, "delta_kv_append_layers") if check else s
 
 
 def full_attn(desc, pt, q, k_pool, v_pool, o, workspace, ws_bytes: int, stream: int = 0, check: bool = True) -> int:

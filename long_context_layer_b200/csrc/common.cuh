@@ -1,6 +1,7 @@
 // Shared device helpers of the DELTA decode kernels (included by delta_attn.cu only).
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -72,6 +73,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
             "r"(smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
+}
+
+// Bulk prefetch of a global range into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ float exp2_approx(float x) {
@@ -155,100 +161,268 @@ struct DecodeParams {
     float* part_o;    // [B][Hq][S][D] unnormalised outputs of each split
     float2* page_ml;  // [B][Hq][max_pages] per-page (max, sum) for delta-layers
     void* o;          // [B][Hq][D] output
-    float2* lse;      // [B][Hq] (max, sum) over the whole context, delta-layers only (else null)
+    int32_t num_clusters;   // clusters along the split dimension (num_splits = cluster size * this)
     int* tickets;     // [B][Hkv] arrival counters of the split CTAs, zero between launches
     int* err;
 };
 
 
-// Epilogue shared by the decode kernels.  mo [NPART][kMaxGroup][D] and mml [NPART][kMaxGroup][2]
-// (in shared memory) hold NPART partial states (base-2 max, sum, unnormalised output) of the
-// G query heads of this CTA.  They are merged into this split's partial in global memory; the
-// last CTA of (b, g) to arrive then merges all splits and writes o (and lse for delta-layers).
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Wait until the grids this one depends on have completed and their writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel in the stream be scheduled (its CTAs still wait in pdl_wait()).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ------------------------------------------------------------------ page lists
+// Logical and physical page of the pages a warp streams, fetched by all 32 lanes at once (one
+// page per lane, so the two dependent loads are paid once per 32 pages) and kept one chunk of
+// 32 pages ahead of use.  Pages that must be skipped get phys = -1 (and raise an error flag).
+struct WarpPages {
+    int lp_a, ph_a;   // chunk `cur`
+    int lp_b, ph_b;   // chunk `cur + 1`
+    int cur;
+};
+
+struct SeqExtent {
+    int n;      // tokens (clamped)
+    int N;      // pages
+    int pbeg;   // first entry of the sequence in page_indices
+    int count;  // items to attend: N, or the selection length
+};
+
+template <typename P>
+__device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int b, int i0, int warp, int nk, int kbase,
+                                            int lane, int& lp, int& ph) {
+    const int k = kbase + lane;
+    lp = -1;
+    ph = -1;
+    if (k >= nk) return;
+    const int i = i0 + warp + k * kWarps;
+    lp = (p.mode == kModeSparse) ? p.sel_pages[size_t(b) * p.sel_stride + i] : i;
+    if (lp < 0 || lp >= ex.N) {
+        atomicOr(p.err, kErrSel);
+        return;
+    }
+    const int64_t x = p.indices[ex.pbeg + lp];
+    if (x < 0 || x >= p.num_phys_pages) {
+        atomicOr(p.err, kErrPage);
+        return;
+    }
+    ph = int(x);
+}
+
+template <typename P>
+__device__ __forceinline__ void pages_init(WarpPages& w, const P& p, const SeqExtent& ex, int b, int i0, int warp,
+                                           int nk, int lane) {
+    w.cur = 0;
+    fetch_pages(p, ex, b, i0, warp, nk, 0, lane, w.lp_a, w.ph_a);
+    fetch_pages(p, ex, b, i0, warp, nk, 32, lane, w.lp_b, w.ph_b);
+}
+
+// Called by all lanes at the top of iteration k (uniform).
+template <typename P>
+__device__ __forceinline__ void pages_advance(WarpPages& w, const P& p, const SeqExtent& ex, int b, int i0, int warp,
+                                              int nk, int lane, int k) {
+    if (k > 0 && (k & 31) == 0) {
+        w.cur = k >> 5;
+        w.lp_a = w.lp_b;
+        w.ph_a = w.ph_b;
+        fetch_pages(p, ex, b, i0, warp, nk, (w.cur + 1) * 32, lane, w.lp_b, w.ph_b);
+    }
+}
+
+// Page k of the warp (all lanes call; k must lie in chunk cur or cur + 1).
+__device__ __forceinline__ void pages_get(const WarpPages& w, int k, int& lp, int& ph) {
+    const bool a = (k >> 5) == w.cur;
+    lp = __shfl_sync(0xffffffffu, a ? w.lp_a : w.lp_b, k & 31);
+    ph = __shfl_sync(0xffffffffu, a ? w.ph_a : w.ph_b, k & 31);
+}
+
+// Tokens and item count of sequence b, validated against the page table (bad values clamped
+// and flagged).
+template <typename P>
+__device__ __forceinline__ SeqExtent seq_extent(const P& p, int b) {
+    SeqExtent ex;
+    int n = p.kv_len[b];
+    ex.pbeg = p.indptr[b];
+    const int npg = p.indptr[b + 1] - ex.pbeg;
+    const int scnt = (p.mode == kModeSparse) ? p.sel_cnt[b] : 0;
+    if (n < 0) n = 0;
+    if (n > npg * kPage || n > p.max_pages * kPage) {
+        if (threadIdx.x == 0) atomicOr(p.err, kErrLen);
+        n = min(max(npg, 0), p.max_pages) * kPage;
+    }
+    ex.n = n;
+    ex.N = (n + kPage - 1) / kPage;
+    ex.count = ex.N;
+    if (p.mode == kModeSparse) {
+        const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
+        ex.count = scnt;
+        if (scnt < 0 || scnt > cap) {
+            if (threadIdx.x == 0) atomicOr(p.err, kErrSel);
+            ex.count = min(max(scnt, 0), cap);
+        }
+    }
+    return ex;
+}
+
+// Epilogue shared by the decode kernels.
+//
+// mo [NPART][kMaxGroup][D] and mml [NPART][kMaxGroup][2] (shared memory) hold NPART partial
+// states (base-2 running max, sum of exponentials, unnormalised output) of the G query heads
+// of this CTA.  The C CTAs of a thread-block cluster cover C consecutive splits of one
+// (sequence, KV head): each reduces its NPART states to one, the cluster merges those through
+// distributed shared memory (every CTA finalises a 1/C slice of the G x D outputs), and
+//   - with one cluster per (sequence, KV head) the slice is the final output;
+//   - with nC > 1 clusters each writes a cluster partial to the workspace, and the last CTA to
+//     arrive (an atomic ticket; nobody waits) merges the nC partials into the output.
+// Floats of the dedicated receive area of the cluster merge (never aliased with pipeline stages,
+// so other CTAs of the cluster may push into it while this CTA is still streaming pages).
+template <int D>
+constexpr int recv_floats() { return kMaxGroup * D + 16 * 4 + 16 * kMaxGroup * 2 + kMaxGroup * 2; }
+
 template <typename T, int D, int G, int NPART>
-__device__ __forceinline__ void split_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
-                                               const float* mml, int b, int g, int split) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
+                                               const float* mml, float* recv, int b, int g) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = int(cluster.num_blocks());
+    const int rank = int(cluster.block_rank());
+    const int cidx = blockIdx.x / C;
+    const int nC = p.num_clusters;
     const int Hq = p.num_q_heads;
     const int h0 = g * G;
-    const int S_ = p.num_splits;
-    for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
-        const int h = idx / D, d = idx % D;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    T* out = reinterpret_cast<T*>(p.o);
+
+    // 1. this CTA's NPART states -> one state, pushed straight into the shared memory of the
+    //    cluster CTA that owns each output element (remote stores need no round trip).  Slices
+    //    are multiples of 4 elements so every push is one 16-byte store.
+    const int total = G * D;
+    const int chunk = (((total + C - 1) / C) + 3) & ~3;
+    float* recv_ml = recv + C * chunk;                                             // [C][G][2]
+    float* cml = recv_ml + C * G * 2;                                              // [G][2] this CTA
+    if (tid < G) {
         float M = -INFINITY;
 #pragma unroll
-        for (int rr = 0; rr < NPART; ++rr) M = fmaxf(M, mml[(rr * kMaxGroup + h) * 2]);
+        for (int rr = 0; rr < NPART; ++rr) M = fmaxf(M, mml[(rr * kMaxGroup + tid) * 2]);
         const float mu = (M == -INFINITY) ? 0.f : M;
-        float L = 0.f, acc = 0.f;
+        float L = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < NPART; ++rr)
+            L = fmaf(exp2_approx(mml[(rr * kMaxGroup + tid) * 2] - mu), mml[(rr * kMaxGroup + tid) * 2 + 1], L);
+        cml[2 * tid] = M;
+        cml[2 * tid + 1] = L;
+    }
+    __syncthreads();
+    if (tid < C * G) {   // this CTA's (max, sum) of head h to cluster rank j
+        const int j = tid / G, h = tid % G;
+        reinterpret_cast<float2*>(cluster.map_shared_rank(recv_ml, j))[rank * G + h] =
+            make_float2(cml[2 * h], cml[2 * h + 1]);
+    }
+    for (int q4 = tid; q4 * 4 < total; q4 += nthr) {
+        const int idx = q4 * 4, h = idx / D, d = idx % D;    // D is a multiple of 4: one head per group
+        const float M = cml[2 * h];
+        const float mu = (M == -INFINITY) ? 0.f : M;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int rr = 0; rr < NPART; ++rr) {
             const float w = exp2_approx(mml[(rr * kMaxGroup + h) * 2] - mu);
-            L = fmaf(w, mml[(rr * kMaxGroup + h) * 2 + 1], L);
-            acc = fmaf(w, mo[(rr * kMaxGroup + h) * D + d], acc);
+            const float4 v = *reinterpret_cast<const float4*>(&mo[(rr * kMaxGroup + h) * D + d]);
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
         }
-        const size_t row = (size_t(b) * Hq + h0 + h) * S_ + split;
-        p.part_o[row * D + d] = acc;
-        if (d == 0) p.part_ml[row] = make_float2(M, L);
+        const int owner = idx / chunk;
+        *reinterpret_cast<float4*>(cluster.map_shared_rank(recv, owner) + rank * chunk + (idx - owner * chunk)) = acc;
     }
+    cluster.sync();   // release/acquire: every pushed value is visible to its owner
 
-    // ---- the last CTA of (b, g) to finish merges the splits; nobody waits for anybody
+    // 2. each CTA merges the C states of its slice from its own shared memory
+    const int e0 = rank * chunk, e1 = min(e0 + chunk, total);
+    for (int e = e0 + tid; e < e1; e += nthr) {
+        const int h = e / D, d = e % D;
+        float M = -INFINITY;
+        for (int j = 0; j < C; ++j) M = fmaxf(M, recv_ml[(j * G + h) * 2]);
+        const float mu = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f, acc = 0.f;
+        for (int j = 0; j < C; ++j) {
+            const float w = exp2_approx(recv_ml[(j * G + h) * 2] - mu);
+            L = fmaf(w, recv_ml[(j * G + h) * 2 + 1], L);
+            acc = fmaf(w, recv[j * chunk + (e - e0)], acc);
+        }
+        if (nC == 1) {
+            out[(size_t(b) * Hq + h0 + h) * D + d] = Elem<T>::from_f(M == -INFINITY ? 0.f : acc / L);
+        } else {
+            const size_t row = (size_t(b) * Hq + h0 + h) * nC + cidx;
+            p.part_o[row * D + d] = acc;
+            if (d == 0) p.part_ml[row] = make_float2(M, L);
+        }
+    }
+    if (nC == 1) return;
+
+    // 3. the last CTA of (b, g) to arrive merges the nC cluster partials
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         const int t = atomicAdd(&p.tickets[b * p.num_kv_heads + g], 1);
-        s_last = (t == S_ - 1);
+        s_last = (t == C * nC - 1);
         if (s_last) p.tickets[b * p.num_kv_heads + g] = 0;   // ready for the next launch
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // Split weights w[h][s] = 2^(m_s - M_h) / L_h staged in shared memory, then every output
-    // element sums its S partials with independent (unrolled) loads.
-    float* sml = reinterpret_cast<float*>(smem);          // [G][S] (max) then weights
-    float* sl = sml + G * S_;                              // [G][S] (sum)
-    float* sML = sl + G * S_;                              // [G][2] (M, L)
-    for (int idx = threadIdx.x; idx < G * S_; idx += kThreads) {
-        const int h = idx / S_, s2 = idx % S_;
-        const float2 ml = __ldcg(&p.part_ml[(size_t(b) * Hq + h0 + h) * S_ + s2]);
+    float* sml = reinterpret_cast<float*>(smem);          // [G][nC] maxima, then weights
+    float* sl = sml + G * nC;                              // [G][nC] sums
+    float* sML = sl + G * nC;                              // [G][2]
+    for (int idx = tid; idx < G * nC; idx += nthr) {
+        const float2 ml = __ldcg(&p.part_ml[(size_t(b) * Hq + h0) * nC + idx]);
         sml[idx] = ml.x;
         sl[idx] = ml.y;
     }
     __syncthreads();
-    for (int h = warp; h < G; h += kWarps) {
+    for (int h = warp; h < G; h += nthr / 32) {
         float M = -INFINITY;
-        for (int s2 = lane; s2 < S_; s2 += 32) M = fmaxf(M, sml[h * S_ + s2]);
+        for (int c = lane; c < nC; c += 32) M = fmaxf(M, sml[h * nC + c]);
 #pragma unroll
         for (int o2 = 16; o2 >= 1; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
         const float mu = (M == -INFINITY) ? 0.f : M;
         float Ls = 0.f;
-        for (int s2 = lane; s2 < S_; s2 += 32) Ls += exp2_approx(sml[h * S_ + s2] - mu) * sl[h * S_ + s2];
+        for (int c = lane; c < nC; c += 32) Ls += exp2_approx(sml[h * nC + c] - mu) * sl[h * nC + c];
 #pragma unroll
         for (int o2 = 16; o2 >= 1; o2 >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o2);
         if (lane == 0) { sML[2 * h] = M; sML[2 * h + 1] = Ls; }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * S_; idx += kThreads) {
-        const int h = idx / S_;
+    for (int idx = tid; idx < G * nC; idx += nthr) {
+        const int h = idx / nC;
         const float M = sML[2 * h], Ls = sML[2 * h + 1];
         sml[idx] = (M == -INFINITY) ? 0.f : exp2_approx(sml[idx] - M) / Ls;
     }
     __syncthreads();
-    T* out = reinterpret_cast<T*>(p.o);
-    for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
-        const int h = idx / D, d = idx % D;
-        const float* po = p.part_o + (size_t(b) * Hq + h0 + h) * S_ * D + d;
-        const float* w = sml + h * S_;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        int s2 = 0;
-        for (; s2 + 4 <= S_; s2 += 4) {
-            a0 = fmaf(w[s2 + 0], __ldcg(po + size_t(s2 + 0) * D), a0);
-            a1 = fmaf(w[s2 + 1], __ldcg(po + size_t(s2 + 1) * D), a1);
-            a2 = fmaf(w[s2 + 2], __ldcg(po + size_t(s2 + 2) * D), a2);
-            a3 = fmaf(w[s2 + 3], __ldcg(po + size_t(s2 + 3) * D), a3);
+    constexpr int J = (G * D + kThreads - 1) / kThreads;   // outputs per thread
+    float a[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) a[j] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < nC; ++c) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int idx = tid + j * kThreads;
+            if (idx < G * D) {
+                const int h = idx / D, d = idx % D;
+                a[j] = fmaf(sml[h * nC + c], __ldcg(p.part_o + ((size_t(b) * Hq + h0 + h) * nC + c) * D + d), a[j]);
+            }
         }
-        for (; s2 < S_; ++s2) a0 = fmaf(w[s2], __ldcg(po + size_t(s2) * D), a0);
-        out[(size_t(b) * Hq + h0 + h) * D + d] = Elem<T>::from_f((a0 + a1) + (a2 + a3));
-        if (p.lse != nullptr && d == 0) p.lse[size_t(b) * Hq + h0 + h] = make_float2(sML[2 * h], sML[2 * h + 1]);
+    }
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int idx = tid + j * kThreads;
+        if (idx < G * D) out[(size_t(b) * Hq + h0 + idx / D) * D + idx % D] = Elem<T>::from_f(a[j]);
     }
 }
 

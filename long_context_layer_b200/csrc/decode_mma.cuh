@@ -64,13 +64,11 @@ struct MmaSmem {
     static constexpr uint32_t kBox = 16 * 128;                // one box: 16 rows x 128 bytes
     static constexpr uint32_t kPage = 2 * kBoxes * kBox;      // K and V of one page, one KV head
     static constexpr size_t kStages = size_t(kWarps) * STAGES * kPage;
-    static constexpr size_t kMerge = size_t(kWarps) * kMaxGroup * (D + 2) * sizeof(float);
-    static constexpr size_t kLast = size_t(kMaxGroup) * kMaxSplits * 3 * sizeof(float) + 64;
-    static constexpr size_t kMain0 = kStages > kMerge ? kStages : kMerge;
-    static constexpr size_t kMain = kMain0 > kLast ? kMain0 : kLast;
+    static constexpr size_t kMerge = size_t(kWarps + 1) * kMaxGroup * (D + 2) * sizeof(float);
+    static constexpr size_t kMain = kStages > kMerge ? kStages : kMerge;
     static constexpr size_t kBars = size_t(kWarps) * STAGES * sizeof(uint64_t);
-    static constexpr size_t kMeta = size_t(kWarps) * STAGES * sizeof(int2);
-    static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kMeta;
+    static constexpr size_t kRecv = size_t(recv_floats<D>()) * sizeof(float);
+    static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kRecv;
 };
 
 template <int D, int G, int STAGES>
@@ -83,7 +81,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     unsigned char* smem =
         smem_raw + ((1024 - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kMain);
-    int2* meta = reinterpret_cast<int2*>(smem + S::kMain + S::kBars);
+    float* recv = reinterpret_cast<float*>(smem + S::kMain + S::kBars);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g4 = lane >> 2, t4 = lane & 3;
@@ -91,27 +89,46 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     const int Hq = p.num_q_heads;
     const int h0 = g * G;
 
-    // ---- sequence extent (validated; bad values are clamped and flagged)
-    int n = p.kv_len[b];
-    const int pbeg = p.indptr[b];
-    const int npg = p.indptr[b + 1] - pbeg;
-    if (n < 0) n = 0;
-    if (n > npg * kPage || n > p.max_pages * kPage) {
-        if (threadIdx.x == 0) atomicOr(p.err, kErrLen);
-        n = min(max(npg, 0), p.max_pages) * kPage;
+    uint64_t* wbar = bars + warp * STAGES;
+    unsigned char* wst = smem + size_t(warp) * STAGES * S::kPage;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&wbar[s], 1);
+        fence_mbar_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
     }
-    const int N = (n + kPage - 1) / kPage;
-    int count = N;
-    if (p.mode == kModeSparse) {
-        count = p.sel_cnt[b];
-        if (count < 0 || count > p.sel_stride || count > p.items_per_split * p.num_splits) {
-            if (threadIdx.x == 0) atomicOr(p.err, kErrSel);
-            count = min(max(count, 0), min(p.sel_stride, p.items_per_split * p.num_splits));
+    __syncwarp();
+    // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
+    // so full and delta layers resolve their pages before waiting for the previous kernel; the
+    // sparse layers' page list is the output of the delta-layer and is read after the wait.
+    SeqExtent ex;
+    int i0 = 0, nk = 0;
+    WarpPages pages;
+    auto setup = [&]() {
+        ex = seq_extent(p, b);
+        i0 = split * p.items_per_split;
+        const int i1 = min(i0 + p.items_per_split, ex.count);
+        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
+        pages_init(pages, p, ex, b, i0, warp, nk, lane);
+    };
+    if (p.mode != kModeSparse) {
+        setup();
+        // Warm L2 with this warp's first pages while the previous kernel drains.  Only the
+        // current token's slot of a pool changes between layers' kernels, and an L2 prefetch is
+        // coherent with later writes, so this is safe before the wait.
+        if (lane < min(STAGES, nk)) {
+            const int ph = pages.ph_a;   // lane j holds page j of the warp
+            if (ph >= 0) {
+                const size_t off = (size_t(ph) * p.num_kv_heads + g) * kPage * D;
+                prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.k_pool) + off, kPage * D * 2);
+                prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.v_pool) + off, kPage * D * 2);
+            }
         }
     }
-    const int i0 = split * p.items_per_split;
-    const int i1 = min(i0 + p.items_per_split, count);
-    const int nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;
+    pdl_wait();      // q, the pools and the selection are written by earlier kernels
+    pdl_trigger();
+    if (p.mode == kModeSparse) setup();
 
     // ---- Q^T fragments (B operand of the QK product): head g4 of the group, dims k*16 + 2*t4 (+8)
     uint32_t qb[KS][2];
@@ -128,35 +145,16 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         }
     }
 
-    uint64_t* wbar = bars + warp * STAGES;
-    int2* wmeta = meta + warp * STAGES;
-    unsigned char* wst = smem + size_t(warp) * STAGES * S::kPage;
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&wbar[s], 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
     const uint64_t policy = evict_first_policy();
-    const int row_base_g = g * kPage;   // row of (page, g) = (phys * Hkv + g) * 16
-
-    auto issue = [&](int k) {   // lane 0 only
+    // all lanes call (the page id is shuffled out of the prefetched list); lane 0 issues
+    auto issue = [&](int k) {
+        int lp, ph;
+        pages_get(pages, k, lp, ph);
+        if (lane != 0) return;
         const int s = k % STAGES;
-        const int i = i0 + warp + k * kWarps;
-        const int lp = (p.mode == kModeSparse) ? p.sel_pages[size_t(b) * p.sel_stride + i] : i;
-        int valid = 0;
-        int64_t phys = -1;
-        if (lp >= 0 && lp < N) {
-            phys = p.indices[pbeg + lp];
-            valid = (phys >= 0 && phys < p.num_phys_pages) ? 1 : 0;
-            if (!valid) atomicOr(p.err, kErrPage);
-        } else {
-            atomicOr(p.err, kErrSel);
-        }
-        wmeta[s] = make_int2(lp, valid);
-        if (valid) {
+        if (ph >= 0) {
             unsigned char* dst = wst + size_t(s) * S::kPage;
-            const int y = int(phys) * p.num_kv_heads * kPage + row_base_g;
+            const int y = (ph * p.num_kv_heads + g) * kPage;   // row of (page, KV head g)
             mbar_expect_tx(&wbar[s], S::kPage);
 #pragma unroll
             for (int nb = 0; nb < S::kBoxes; ++nb) {
@@ -164,11 +162,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
                 tma_load_2d(dst + (S::kBoxes + nb) * S::kBox, &tmap_v, nb * 64, y, &wbar[s], policy);
             }
         } else {
-            mbar_arrive(&wbar[s]);
+            mbar_arrive(&wbar[s]);   // completes the phase with no data; the page is skipped
         }
     };
-    if (lane == 0)
-        for (int k = 0; k < min(STAGES, nk); ++k) issue(k);
+    for (int k = 0; k < min(STAGES, nk); ++k) issue(k);
 
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2*t4, 2*t4+1
     float acc[KS][4];
@@ -184,70 +181,120 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     bool failed = false;
     int consumed = 0;
 
-    for (int k = 0; k < nk; ++k) {
-        const int s = k % STAGES;
-        if (!mbar_wait(&wbar[s], (k / STAGES) & 1)) {
+    // S^T (16 tokens x 8 heads) of the page in stage s; masked tokens get -inf.  Two accumulator
+    // chains (even / odd k-steps) halve the dependent MMA chain.
+    auto qk_page = [&](int s, int tv, float (&sc)[4]) {
+        const uint32_t kbase = smem_addr(wst + size_t(s) * S::kPage);
+        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const int chunk = kk * 2 + k_sub;               // 16-byte chunk of the row (0..D/8-1)
+            const uint32_t addr = kbase + (chunk >> 3) * S::kBox + k_row * 128 + (((chunk & 7) ^ (k_row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(addr, a0, a1, a2, a3);
+            if (kk & 1) mma_bf16_16816(c1, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+            else mma_bf16_16816(c0, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+        }
+        // base-2 logits; tokens g4 and g4+8, heads 2*t4 and 2*t4+1
+        const bool ok0 = g4 < tv, ok1 = g4 + 8 < tv;
+        sc[0] = ok0 ? (c0[0] + c1[0]) * p.qscale : -INFINITY;
+        sc[1] = ok0 ? (c0[1] + c1[1]) * p.qscale : -INFINITY;
+        sc[2] = ok1 ? (c0[2] + c1[2]) * p.qscale : -INFINITY;
+        sc[3] = ok1 ? (c0[3] + c1[3]) * p.qscale : -INFINITY;
+    };
+    // Delta-layers: page partials from the unrounded probabilities (max logit, sum of 2^(s - max))
+    auto page_partials = [&](const float (&sc)[4], int lp) {
+        float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        float e0 = exp2_approx(sc[0] - mx0) + exp2_approx(sc[2] - mx0);
+        float e1 = exp2_approx(sc[1] - mx1) + exp2_approx(sc[3] - mx1);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            e0 += __shfl_xor_sync(0xffffffffu, e0, o);
+            e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+        }
+        const int hA = 2 * t4, hB = 2 * t4 + 1;
+        if (g4 == 0 && hA < G) p.page_ml[(size_t(b) * Hq + h0 + hA) * p.max_pages + lp] = make_float2(mx0, e0);
+        if (g4 == 0 && hB < G) p.page_ml[(size_t(b) * Hq + h0 + hB) * p.max_pages + lp] = make_float2(mx1, e1);
+    };
+    // tokens past the end of the context: zero their V rows (they may hold non-finite bytes)
+    auto zero_tail = [&](int s, int tv) {
+        uint4* vz = reinterpret_cast<uint4*>(wst + size_t(s) * S::kPage + S::kBoxes * S::kBox);
+        const int per_box = (kPage - tv) * 8;
+        for (int c = lane; c < S::kBoxes * per_box; c += 32) {
+            const int box = c / per_box, rem = c % per_box;
+            vz[box * (S::kBox / 16) + (tv + rem / 8) * 8 + (rem % 8)] = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+    };
+    // O^T += V^T . P^T for the page in stage s
+    auto pv_page = [&](int s, uint32_t pb0, uint32_t pb1) {
+        const uint32_t vbase = smem_addr(wst + size_t(s) * S::kPage) + S::kBoxes * S::kBox;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            const int chunk = mt * 2 + v_sub;
+            const uint32_t addr = vbase + (chunk >> 3) * S::kBox + v_row * 128 + (((chunk & 7) ^ (v_row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+            mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+    };
+
+    // Pages are taken two at a time: their QK products, one softmax update and their PV
+    // products are independent chains the scheduler interleaves.
+    for (int k = 0; k < nk; k += 2) {
+        pages_advance(pages, p, ex, b, i0, warp, nk, lane, k);
+        const bool two = k + 1 < nk;
+        const int sA = k % STAGES, sB = (k + 1) % STAGES;
+        if (!mbar_wait(&wbar[sA], (k / STAGES) & 1) || (two && !mbar_wait(&wbar[sB], ((k + 1) / STAGES) & 1))) {
             if (lane == 0) atomicOr(p.err, kErrTimeout);
             failed = true;
             break;
         }
-        consumed = k + 1;
-        const int2 mt_ = wmeta[s];
+        consumed = k + (two ? 2 : 1);
+        int lpA, phA, lpB = -1, phB = -1;
+        pages_get(pages, k, lpA, phA);
+        if (two) pages_get(pages, k + 1, lpB, phB);
+        const bool vA = phA >= 0, vB = phB >= 0;
+        const int tvA = vA ? min(kPage, ex.n - lpA * kPage) : 0;
+        const int tvB = vB ? min(kPage, ex.n - lpB * kPage) : 0;
+        float scA[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float scB[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (vA) qk_page(sA, tvA, scA);
+        if (vB) qk_page(sB, tvB, scB);
         bool zeroed = false;
-        if (mt_.y) {
-            const int lp = mt_.x;
-            const int tv = min(kPage, n - lp * kPage);
-            const uint32_t kbase = smem_addr(wst + size_t(s) * S::kPage);
-            const uint32_t vbase = kbase + S::kBoxes * S::kBox;
-            // S^T = K . Q^T
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                const int chunk = kk * 2 + k_sub;               // 16-byte chunk of the row (0..D/8-1)
-                const uint32_t addr = kbase + (chunk >> 3) * S::kBox + k_row * 128 + (((chunk & 7) ^ (k_row & 7)) << 4);
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4(addr, a0, a1, a2, a3);
-                mma_bf16_16816(sc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+        if (vA || vB) {
+            if (p.mode == kModeDelta) {
+                if (vA) page_partials(scA, lpA);
+                if (vB) page_partials(scB, lpB);
             }
-            // base-2 logits; tokens g4 and g4+8, heads 2*t4 and 2*t4+1
-            const bool ok0 = g4 < tv, ok1 = g4 + 8 < tv;
-            sc[0] = ok0 ? sc[0] * p.qscale : -INFINITY;
-            sc[1] = ok0 ? sc[1] * p.qscale : -INFINITY;
-            sc[2] = ok1 ? sc[2] * p.qscale : -INFINITY;
-            sc[3] = ok1 ? sc[3] * p.qscale : -INFINITY;
-            float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+            float mx0 = fmaxf(fmaxf(scA[0], scA[2]), fmaxf(scB[0], scB[2]));
+            float mx1 = fmaxf(fmaxf(scA[1], scA[3]), fmaxf(scB[1], scB[3]));
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
             }
-            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);   // mx is finite: tv >= 1
+            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);   // finite: a valid token exists
             const float al0 = exp2_approx(m_run[0] - mn0), al1 = exp2_approx(m_run[1] - mn1);
-            const uint32_t x0 = pack_bf16(exp2_approx(sc[0] - mn0), exp2_approx(sc[1] - mn1));
-            const uint32_t x1 = pack_bf16(exp2_approx(sc[2] - mn0), exp2_approx(sc[3] - mn1));
-            float p0, p1, p2, p3;
-            unpack_bf16x2(x0, p0, p1);
-            unpack_bf16x2(x1, p2, p3);
-            float rs0 = p0 + p2, rs1 = p1 + p3;
+            const uint32_t xa0 = pack_bf16(exp2_approx(scA[0] - mn0), exp2_approx(scA[1] - mn1));
+            const uint32_t xa1 = pack_bf16(exp2_approx(scA[2] - mn0), exp2_approx(scA[3] - mn1));
+            const uint32_t xb0 = pack_bf16(exp2_approx(scB[0] - mn0), exp2_approx(scB[1] - mn1));
+            const uint32_t xb1 = pack_bf16(exp2_approx(scB[2] - mn0), exp2_approx(scB[3] - mn1));
+            float p0, p1, p2, p3, q0, q1, q2, q3;
+            unpack_bf16x2(xa0, p0, p1);
+            unpack_bf16x2(xa1, p2, p3);
+            unpack_bf16x2(xb0, q0, q1);
+            unpack_bf16x2(xb1, q2, q3);
+            float rs0 = (p0 + p2) + (q0 + q2), rs1 = (p1 + p3) + (q1 + q3);
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
                 rs0 += __shfl_xor_sync(0xffffffffu, rs0, o);
                 rs1 += __shfl_xor_sync(0xffffffffu, rs1, o);
-            }
-            if (p.mode == kModeDelta) {
-                // page partials from the unrounded probabilities: max logit and sum of 2^(s - max)
-                float e0 = exp2_approx(sc[0] - mx0) + exp2_approx(sc[2] - mx0);
-                float e1 = exp2_approx(sc[1] - mx1) + exp2_approx(sc[3] - mx1);
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    e0 += __shfl_xor_sync(0xffffffffu, e0, o);
-                    e1 += __shfl_xor_sync(0xffffffffu, e1, o);
-                }
-                const int hA = 2 * t4, hB = 2 * t4 + 1;
-                if (g4 == 0 && hA < G)
-                    p.page_ml[(size_t(b) * Hq + h0 + hA) * p.max_pages + lp] = make_float2(mx0, e0);
-                if (g4 == 0 && hB < G)
-                    p.page_ml[(size_t(b) * Hq + h0 + hB) * p.max_pages + lp] = make_float2(mx1, e1);
             }
             l_run[0] = l_run[0] * al0 + rs0;
             l_run[1] = l_run[1] * al1 + rs1;
@@ -260,35 +307,18 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
                 acc[mt][2] *= al0;
                 acc[mt][3] *= al1;
             }
-            const uint32_t pb0 = movmatrix_trans(x0), pb1 = movmatrix_trans(x1);
-            if (tv < kPage) {
-                // tokens past the end of the context: zero their V rows (they may hold non-finite bytes)
-                uint4* vz = reinterpret_cast<uint4*>(wst + size_t(s) * S::kPage + S::kBoxes * S::kBox);
-                const int nchunks = S::kBoxes * (kPage - tv) * 8;
-                for (int c = lane; c < nchunks; c += 32) {
-                    const int box = c / ((kPage - tv) * 8), rem = c % ((kPage - tv) * 8);
-                    vz[box * (S::kBox / 16) + (tv + rem / 8) * 8 + (rem % 8)] = make_uint4(0, 0, 0, 0);
-                }
-                __syncwarp();
-                zeroed = true;
-            }
-            // O^T += V^T . P^T
-#pragma unroll
-            for (int mt = 0; mt < KS; ++mt) {
-                const int chunk = mt * 2 + v_sub;
-                const uint32_t addr = vbase + (chunk >> 3) * S::kBox + v_row * 128 + (((chunk & 7) ^ (v_row & 7)) << 4);
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4_trans(addr, a0, a1, a2, a3);
-                mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
-            }
+            if (vA && tvA < kPage) { zero_tail(sA, tvA); zeroed = true; }
+            if (vB && tvB < kPage) { zero_tail(sB, tvB); zeroed = true; }
+            if (vA) pv_page(sA, movmatrix_trans(xa0), movmatrix_trans(xa1));
+            if (vB) pv_page(sB, movmatrix_trans(xb0), movmatrix_trans(xb1));
         }
         __syncwarp();
-        if (lane == 0 && k + STAGES < nk) {
-            if (zeroed) fence_proxy_async_smem();
-            issue(k + STAGES);
-        }
+        if (zeroed && lane == 0) fence_proxy_async_smem();
+        if (k + STAGES < nk) issue(k + STAGES);
+        if (two && k + 1 + STAGES < nk) issue(k + 1 + STAGES);
     }
     if (failed) {
+        // drain this warp's copies still in flight (bounded) before shared memory is released
         for (int k = consumed + 1; k < min(consumed + STAGES, nk); ++k) mbar_wait(&wbar[k % STAGES], (k / STAGES) & 1);
     }
 
@@ -311,7 +341,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         mml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 1] = l_run[1];
     }
     __syncthreads();
-    split_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo, mml, b, g, split);
+    merge_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo, mml, recv, b, g);
 }
 
 }  // namespace delta

@@ -12,9 +12,10 @@ struct DecodeSmem {
     static constexpr size_t kBars = size_t(kWarps) * STAGES * sizeof(uint64_t);
     static constexpr size_t kPbuf = size_t(kWarps) * 2 * 8 * kMaxGroup * sizeof(float);
     static constexpr size_t kAbuf = size_t(kWarps) * 2 * kMaxGroup * sizeof(float);
-    static constexpr size_t kMerge = size_t(kWarps) * 2 * kMaxGroup * (D + 2) * sizeof(float);
+    static constexpr size_t kMerge = size_t(kWarps * 2 + 1) * kMaxGroup * (D + 2) * sizeof(float);
     static constexpr size_t kMain = kStages > kMerge ? kStages : kMerge;
-    static constexpr size_t kBytes = kMain + kBars + kPbuf + kAbuf;
+    static constexpr size_t kRecv = size_t(recv_floats<D>()) * sizeof(float);
+    static constexpr size_t kBytes = kMain + kBars + kPbuf + kAbuf + kRecv;
 };
 
 template <typename T, int D, int G, int STAGES>
@@ -29,6 +30,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kMain);
     float* pbuf = reinterpret_cast<float*>(smem + S::kMain + S::kBars);
     float* abuf = pbuf + kWarps * 2 * 8 * kMaxGroup;
+    float* recv = reinterpret_cast<float*>(smem + S::kMain + S::kBars + S::kPbuf + S::kAbuf);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int half = lane >> 4, hl = lane & 15;
@@ -36,27 +38,32 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     const int Hq = p.num_q_heads;
     const int h0 = g * G;
 
-    // ---- sequence extent (validated; bad values are clamped and flagged)
-    int n = p.kv_len[b];
-    const int pbeg = p.indptr[b];
-    const int npg = p.indptr[b + 1] - pbeg;
-    if (n < 0) n = 0;
-    if (n > npg * kPage || n > p.max_pages * kPage) {   // beyond the sequence's pages or the stated bound
-        if (threadIdx.x == 0) atomicOr(p.err, kErrLen);
-        n = min(max(npg, 0), p.max_pages) * kPage;
+    uint64_t* wbar = bars + warp * STAGES;
+    T* wst = stages + size_t(warp) * STAGES * 2 * PE;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&wbar[s], 1);
+        fence_mbar_init();
     }
-    const int N = (n + kPage - 1) / kPage;
-    int count = N;
-    if (p.mode == kModeSparse) {
-        count = p.sel_cnt[b];
-        if (count < 0 || count > p.sel_stride || count > p.items_per_split * p.num_splits) {
-            if (threadIdx.x == 0) atomicOr(p.err, kErrSel);
-            count = min(max(count, 0), min(p.sel_stride, p.items_per_split * p.num_splits));
-        }
-    }
-    const int i0 = split * p.items_per_split;
-    const int i1 = min(i0 + p.items_per_split, count);
-    const int nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;  // pages of this warp
+    __syncwarp();
+    // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
+    // so full and delta layers resolve their pages before waiting for the previous kernel; the
+    // sparse layers' page list is the output of the delta-layer and is read after the wait.
+    SeqExtent ex;
+    int i0 = 0, nk = 0;
+    WarpPages pages;
+    auto setup = [&]() {
+        ex = seq_extent(p, b);
+        i0 = split * p.items_per_split;
+        const int i1 = min(i0 + p.items_per_split, ex.count);
+        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
+        pages_init(pages, p, ex, b, i0, warp, nk, lane);
+    };
+    if (p.mode != kModeSparse) setup();
+    pdl_wait();      // q, the pools and the selection are written by earlier kernels
+    pdl_trigger();
+    if (p.mode == kModeSparse) setup();
+    const int n = ex.n;
 
     // ---- queries of the group, pre-scaled into base-2 logits
     float q[G][DS];
@@ -70,45 +77,27 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         }
     }
 
-    uint64_t* wbar = bars + warp * STAGES;
-    T* wst = stages + size_t(warp) * STAGES * 2 * PE;
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(&wbar[s], 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-
     const T* kpool = reinterpret_cast<const T*>(p.k_pool);
     const T* vpool = reinterpret_cast<const T*>(p.v_pool);
     const uint64_t policy = evict_first_policy();
 
-    // logical page of the warp's k-th item and its physical page; false if it must be skipped
-    auto resolve = [&](int k, int& lp, int64_t& phys) -> bool {
-        const int i = i0 + warp + k * kWarps;
-        lp = (p.mode == kModeSparse) ? p.sel_pages[size_t(b) * p.sel_stride + i] : i;
-        if (lp < 0 || lp >= N) return false;
-        phys = p.indices[pbeg + lp];
-        return phys >= 0 && phys < p.num_phys_pages;
-    };
-    auto issue = [&](int k) {  // lane 0 only
-        int lp;
-        int64_t phys;
+    // all lanes call (the page id is shuffled out of the prefetched list); lane 0 issues
+    auto issue = [&](int k) {
+        int lp, ph;
+        pages_get(pages, k, lp, ph);
+        if (lane != 0) return;
         const int s = k % STAGES;
-        if (resolve(k, lp, phys)) {
+        if (ph >= 0) {
             T* dst = wst + size_t(s) * 2 * PE;
-            const size_t off = (size_t(phys) * p.num_kv_heads + g) * PE;
+            const size_t off = (size_t(ph) * p.num_kv_heads + g) * PE;
             mbar_expect_tx(&wbar[s], 2 * S::kChunk);
             bulk_load(dst, kpool + off, S::kChunk, &wbar[s], policy);
             bulk_load(dst + PE, vpool + off, S::kChunk, &wbar[s], policy);
         } else {
-            atomicOr(p.err, (lp < 0 || lp >= N) ? kErrSel : kErrPage);
             mbar_arrive(&wbar[s]);  // completes the phase with no data; consumers skip the page
         }
     };
-
-    if (lane == 0)
-        for (int k = 0; k < min(STAGES, nk); ++k) issue(k);
+    for (int k = 0; k < min(STAGES, nk); ++k) issue(k);
 
     float m_run = -INFINITY, l_run = 0.f;  // running state of head (hl & (GP-1)) of this half
     float o[G][DS];
@@ -123,6 +112,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     int consumed = 0;
 
     for (int k = 0; k < nk; ++k) {
+        pages_advance(pages, p, ex, b, i0, warp, nk, lane, k);
         const int s = k % STAGES;
         if (!mbar_wait(&wbar[s], (k / STAGES) & 1)) {
             if (lane == 0) atomicOr(p.err, kErrTimeout);
@@ -130,9 +120,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
             break;
         }
         consumed = k + 1;
-        int lp;
-        int64_t phys;
-        if (resolve(k, lp, phys)) {
+        int lp, ph;
+        pages_get(pages, k, lp, ph);
+        if (ph >= 0) {
             const T* Ks = wst + size_t(s) * 2 * PE;
             const T* Vs = Ks + PE;
             const int tv = min(kPage, n - lp * kPage);     // valid tokens of this page
@@ -218,7 +208,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
             }
         }
         __syncwarp();
-        if (lane == 0 && k + STAGES < nk) issue(k + STAGES);
+        if (k + STAGES < nk) issue(k + STAGES);
     }
     if (failed) {
         // drain this warp's copies still in flight (bounded) before shared memory is released
@@ -239,7 +229,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         mml[(r * kMaxGroup + hl) * 2 + 1] = l_run;
     }
     __syncthreads();
-    split_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, b, g, split);
+    merge_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, recv, b, g);
 }
 
 }  // namespace delta

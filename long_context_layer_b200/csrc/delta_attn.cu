@@ -35,6 +35,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -44,7 +45,8 @@
 namespace delta {
 
 // ------------------------------------------------------------------ host side
-constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB each for D = 128)
+constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB each for D = 128), 2 CTAs/SM
+constexpr int kMmaStagesDeep = 6;  // when the whole grid fits one CTA per SM: twice the pages in flight
 constexpr int kMaxQHeadsSelect = 256;
 
 struct WsLayout {
@@ -93,23 +95,53 @@ int ctas_per_sm(int dtype, int D) {
     return c < 1 ? 1 : (c > 8 ? 8 : c);
 }
 
-// Split count: one full wave of CTAs over the GPU, at least 4 pages per CTA (one per warp).
-int num_splits_for(int dtype, int D, int batch, int Hkv, int items) {
-    if (items <= 0) return 1;
-    const int slots = device_sm_count() * ctas_per_sm(dtype, D);
+// Split plan: about one full wave of CTAs over the GPU, at least 4 pages per CTA (one per
+// warp).  Up to 16 splits form one thread-block cluster; more are grouped into clusters of 8
+// whose partials meet in the workspace.
+struct SplitPlan {
+    int cluster, clusters;
+    bool deep;   // one CTA per SM: the deeper-pipelined tensor-core variant
+    int splits() const { return cluster * clusters; }
+};
+
+int split_target_per_sm(int dtype, int D) {
+    static int override_ = -2;
+    if (override_ == -2) {
+        const char* e = getenv("DELTA_CTAS_PER_SM");   // tuning override for sweeps
+        override_ = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
+    }
+    return override_ > 0 ? override_ : ctas_per_sm(dtype, D);
+}
+
+// About one wave of CTAs, at least 4 pages per CTA (one per warp).  The splits of one (sequence,
+// KV head) form clusters of at most 16 CTAs that merge through distributed shared memory; only
+// when more than 31 splits pay off do several clusters meet in the workspace.
+SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
+    if (items <= 0) return {1, 1, false};
+    const int sms = device_sm_count();
+    const int slots = sms * split_target_per_sm(dtype, D);
     const int units = batch * Hkv;
     int s = slots / (units > 0 ? units : 1);
     const int cap = (items + kWarps - 1) / kWarps;
     if (s > cap) s = cap;
     if (s > kMaxSplits) s = kMaxSplits;
+    static int max_splits = -2;
+    if (max_splits == -2) {
+        const char* e = getenv("DELTA_MAX_SPLITS");   // tuning override for sweeps
+        max_splits = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
+    }
+    if (max_splits > 0 && s > max_splits) s = max_splits;
     if (s < 1) s = 1;
-    const int ips = (items + s - 1) / s;
-    return (items + ips - 1) / ips;
+    SplitPlan pl;
+    pl.cluster = s < 16 ? s : 16;
+    pl.clusters = s / pl.cluster;
+    pl.deep = dtype == DELTA_BF16 && int64_t(units) * pl.splits() <= sms;
+    return pl;
 }
 
 WsLayout ws_layout(const delta_desc* d, int batch, int max_pages) {
     WsLayout w{};
-    const int S = num_splits_for(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages);
+    const int S = plan_splits(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages).clusters;
     const size_t rows = size_t(batch) * d->num_q_heads;
     size_t off = 0;
     w.err = off;        off += align256(64);
@@ -195,26 +227,175 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const delta_desc* d) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int D, int G>
-delta_status launch_simt_g(const DecodeParams& prm, int batch, int Hkv, cudaStream_t st) {
-    constexpr int STAGES = simt_stages(int(sizeof(T)), D);
-    using Sm = DecodeSmem<T, D, STAGES>;
-    auto kern = decode_kernel<T, D, G, STAGES>;
-    static int configured[64] = {0};
-    if (!set_smem_once(kern, Sm::kBytes, configured)) return DELTA_ERR_CUDA;
-    kern<<<dim3(prm.num_splits, Hkv, batch), kThreads, Sm::kBytes, st>>>(prm);
+// ---- kernel selection and cluster occupancy
+template <int D, int G>
+const void* mma_ptr(bool deep, size_t* smem) {
+    if (deep) {
+        *smem = MmaSmem<D, kMmaStagesDeep>::kBytes;
+        return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStagesDeep>);
+    }
+    *smem = MmaSmem<D, kMmaStages>::kBytes;
+    return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStages>);
+}
+template <int D, int G>
+const void* simt_ptr(size_t* smem) {
+    constexpr int STAGES = simt_stages(4, D);
+    *smem = DecodeSmem<float, D, STAGES>::kBytes;
+    return reinterpret_cast<const void*>(decode_kernel<float, D, G, STAGES>);
+}
+#define DELTA_G_PTR(G, CALL)  \
+    switch (G) {               \
+        case 1: return CALL(1); \
+        case 2: return CALL(2); \
+        case 3: return CALL(3); \
+        case 4: return CALL(4); \
+        case 5: return CALL(5); \
+        case 6: return CALL(6); \
+        case 7: return CALL(7); \
+        case 8: return CALL(8); \
+        default: return nullptr; \
+    }
+const void* decode_ptr(int dtype, int D, int G, bool deep, size_t* smem) {
+    if (dtype == DELTA_BF16) {
+        if (D == 128) {
+#define CALL(g) mma_ptr<128, g>(deep, smem)
+            DELTA_G_PTR(G, CALL)
+#undef CALL
+        }
+#define CALL(g) mma_ptr<64, g>(deep, smem)
+        DELTA_G_PTR(G, CALL)
+#undef CALL
+    }
+    if (D == 128) {
+#define CALL(g) simt_ptr<128, g>(smem)
+        DELTA_G_PTR(G, CALL)
+#undef CALL
+    }
+#define CALL(g) simt_ptr<64, g>(smem)
+    DELTA_G_PTR(G, CALL)
+#undef CALL
+}
+
+// One-time per-device attributes of a decode kernel (shared-memory limit, cluster sizes > 8).
+bool configure_kernel(const void* func, size_t smem) {
+    constexpr int kSlots = 256;
+    static const void* done_fn[64][kSlots];
+    const int dev = current_device();
+    if (dev < 0) return false;
+    int i = 0;
+    for (; i < kSlots && done_fn[dev][i] != nullptr; ++i)
+        if (done_fn[dev][i] == func) return true;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return false;
+    if (i < kSlots) done_fn[dev][i] = func;
+    return true;
+}
+
+// Clusters of `cluster` CTAs of this kernel that can be resident at once (cached per device).
+int max_active_clusters(const void* func, size_t smem, int cluster) {
+    constexpr int kSlots = 512;
+    struct Entry { const void* fn; int cluster; int n; };
+    static Entry cache[64][kSlots];
+    const int dev = current_device();
+    if (dev < 0) return 1;
+    int i = 0;
+    for (; i < kSlots && cache[dev][i].fn != nullptr; ++i)
+        if (cache[dev][i].fn == func && cache[dev][i].cluster == cluster) return cache[dev][i].n;
+    if (!configure_kernel(func, smem)) return 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster, 1, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, func, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1;
+    }
+    if (i < kSlots) cache[dev][i] = {func, cluster, n};
+    return n;
+}
+
+// Shrink a split plan until all its clusters are resident in one wave (when possible).
+SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units) {
+    for (;;) {
+        size_t smem = 0;
+        const void* fn = decode_ptr(dtype, D, G, pl.deep, &smem);
+        if (fn == nullptr) return pl;
+        const int maxc = max_active_clusters(fn, smem, pl.cluster);
+        if (int64_t(units) * pl.clusters <= maxc) return pl;
+        if (pl.clusters > 1) {
+            pl.clusters = maxc / units > 1 ? maxc / units : 1;
+            continue;
+        }
+        if (pl.cluster == 1) return pl;   // more units than resident clusters: several waves
+        pl.cluster = (pl.cluster + 1) / 2;
+    }
+}
+
+// Launch with programmatic dependent launch: the kernel may be scheduled while the previous
+// kernel of the stream drains; it waits for it in pdl_wait() before touching global memory.
+template <typename K, typename... Args>
+delta_status launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) return DELTA_ERR_CUDA;
     return launch_status();
 }
 
-template <int D, int G>
-delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const CUtensorMap& mv, int batch, int Hkv,
-                          cudaStream_t st) {
-    using Sm = MmaSmem<D, kMmaStages>;
-    auto kern = decode_mma_kernel<D, G, kMmaStages>;
-    static int configured[64] = {0};
-    if (!set_smem_once(kern, Sm::kBytes, configured)) return DELTA_ERR_CUDA;
-    kern<<<dim3(prm.num_splits, Hkv, batch), kThreads, Sm::kBytes, st>>>(prm, mk, mv);
+// Launch a decode kernel as clusters of `cluster` CTAs along the split dimension.
+template <typename K, typename... Args>
+delta_status launch_clustered(K kern, size_t smem, const DecodeParams& prm, int cluster, int batch, int Hkv,
+                              cudaStream_t st, Args... args) {
+    if (!configure_kernel(reinterpret_cast<const void*>(kern), smem)) return DELTA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.num_splits, Hkv, batch);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, prm, args...) != cudaSuccess) return DELTA_ERR_CUDA;
     return launch_status();
+}
+
+template <typename T, int D, int G>
+delta_status launch_simt_g(const DecodeParams& prm, int cluster, int batch, int Hkv, cudaStream_t st) {
+    constexpr int STAGES = simt_stages(int(sizeof(T)), D);
+    return launch_clustered(decode_kernel<T, D, G, STAGES>, DecodeSmem<T, D, STAGES>::kBytes, prm, cluster, batch, Hkv,
+                            st);
+}
+
+template <int D, int G>
+delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const CUtensorMap& mv, int cluster,
+                          bool deep, int batch, int Hkv, cudaStream_t st) {
+    if (deep)
+        return launch_clustered(decode_mma_kernel<D, G, kMmaStagesDeep>, MmaSmem<D, kMmaStagesDeep>::kBytes, prm,
+                                cluster, batch, Hkv, st, mk, mv);
+    return launch_clustered(decode_mma_kernel<D, G, kMmaStages>, MmaSmem<D, kMmaStages>::kBytes, prm, cluster, batch,
+                            Hkv, st, mk, mv);
 }
 
 #define DELTA_G_SWITCH(G, CALL) \
@@ -230,27 +411,28 @@ delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const 
         default: return DELTA_ERR_UNSUPPORTED; \
     }
 
-delta_status launch_decode(const delta_desc* d, const DecodeParams& prm, int batch, cudaStream_t st) {
+delta_status launch_decode(const delta_desc* d, const DecodeParams& prm, int cluster, bool deep, int batch,
+                           cudaStream_t st) {
     const int Hkv = d->num_kv_heads, G = d->num_q_heads / Hkv;
     if (d->dtype == DELTA_BF16) {
         CUtensorMap mk, mv;
         if (!make_pool_map(&mk, prm.k_pool, d) || !make_pool_map(&mv, prm.v_pool, d)) return DELTA_ERR_CUDA;
         if (d->head_dim == 128) {
-#define CALL(g) launch_mma_g<128, g>(prm, mk, mv, batch, Hkv, st)
+#define CALL(g) launch_mma_g<128, g>(prm, mk, mv, cluster, deep, batch, Hkv, st)
             DELTA_G_SWITCH(G, CALL)
 #undef CALL
         } else {
-#define CALL(g) launch_mma_g<64, g>(prm, mk, mv, batch, Hkv, st)
+#define CALL(g) launch_mma_g<64, g>(prm, mk, mv, cluster, deep, batch, Hkv, st)
             DELTA_G_SWITCH(G, CALL)
 #undef CALL
         }
     }
     if (d->head_dim == 128) {
-#define CALL(g) launch_simt_g<float, 128, g>(prm, batch, Hkv, st)
+#define CALL(g) launch_simt_g<float, 128, g>(prm, cluster, batch, Hkv, st)
         DELTA_G_SWITCH(G, CALL)
 #undef CALL
     }
-#define CALL(g) launch_simt_g<float, 64, g>(prm, batch, Hkv, st)
+#define CALL(g) launch_simt_g<float, 64, g>(prm, cluster, batch, Hkv, st)
     DELTA_G_SWITCH(G, CALL)
 #undef CALL
 }
@@ -289,7 +471,9 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     const int D = d->head_dim, Hq = d->num_q_heads, Hkv = d->num_kv_heads;
     int items = pt->max_pages_per_seq;
     if (mode == kModeSparse && sel_stride_in < items) items = sel_stride_in;
-    const int S = num_splits_for(d->dtype, D, pt->batch, Hkv, items);
+    const SplitPlan plan = fit_plan(plan_splits(d->dtype, D, pt->batch, Hkv, items), d->dtype, D, Hq / Hkv,
+                                    pt->batch * Hkv);
+    const int S = plan.splits();
     unsigned char* base = static_cast<unsigned char*>(ws);
 
     DecodeParams prm{};
@@ -316,11 +500,11 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.page_ml = reinterpret_cast<float2*>(base + L.page_ml);
     prm.err = reinterpret_cast<int*>(base + L.err);
     prm.o = o;
-    prm.lse = nullptr;
+    prm.num_clusters = plan.clusters;
     prm.tickets = reinterpret_cast<int*>(base + L.tickets);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    s = launch_decode(d, prm, pt->batch, st);
+    s = launch_decode(d, prm, plan.cluster, plan.deep, pt->batch, st);
     if (s != DELTA_OK || mode != kModeDelta) return s;
 
     SelectParams sp2{};
@@ -340,8 +524,8 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     static int configured[64] = {0};
     if (!set_smem_once(score_select_kernel, size_t(kMaxSelectPages) * sizeof(uint32_t), configured))
         return DELTA_ERR_CUDA;
-    score_select_kernel<<<pt->batch, kSelectThreads, size_t(pt->max_pages_per_seq) * sizeof(uint32_t), st>>>(sp2);
-    return launch_status();
+    return launch_pdl(score_select_kernel, dim3(pt->batch), dim3(kSelectThreads),
+                      size_t(pt->max_pages_per_seq) * sizeof(uint32_t), st, sp2);
 }
 
 }  // namespace delta
@@ -382,11 +566,38 @@ delta_status delta_kv_append(const delta_desc* desc, const delta_page_table* pt,
     // kv_append has no workspace to flag errors in: an out-of-range page is skipped, and the
     // attention call that follows on the same page table flags it.
     const int row_vecs = desc->head_dim * elem_bytes(desc->dtype) / 16;
-    kv_append_kernel<<<dim3(pt->batch, desc->num_kv_heads), 32, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_pool),
-        static_cast<uint4*>(v_pool), pt->page_indptr, pt->page_indices, pt->kv_len, desc->num_kv_heads, row_vecs,
-        desc->num_phys_pages);
-    return launch_status();
+    return launch_pdl(kv_append_kernel, dim3(pt->batch, desc->num_kv_heads), dim3(32), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<const uint4*>(k_new),
+                      static_cast<const uint4*>(v_new), static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool),
+                      pt->page_indptr, pt->page_indices, pt->kv_len, desc->num_kv_heads, row_vecs,
+                      desc->num_phys_pages);
+}
+
+delta_status delta_kv_append_layers(const delta_desc* desc, const delta_page_table* pt, int32_t num_layers,
+                                    const void* const* k_new, const void* const* v_new, void* const* k_pools,
+                                    void* const* v_pools, void* stream) {
+    delta_status s = check_desc(desc);
+    if (s != DELTA_OK) return s;
+    s = check_pt(pt);
+    if (s != DELTA_OK) return s;
+    if (num_layers < 0 || num_layers > kMaxAppendLayers) return num_layers < 0 ? DELTA_ERR_INVALID_ARG : DELTA_ERR_UNSUPPORTED;
+    if (pt->batch == 0 || num_layers == 0) return DELTA_OK;
+    if (k_new == nullptr || v_new == nullptr || k_pools == nullptr || v_pools == nullptr) return DELTA_ERR_INVALID_ARG;
+    AppendLayers a = {};
+    for (int l = 0; l < num_layers; ++l) {
+        if (k_new[l] == nullptr || v_new[l] == nullptr || k_pools[l] == nullptr || v_pools[l] == nullptr)
+            return DELTA_ERR_INVALID_ARG;
+        if (!aligned16(k_new[l]) || !aligned16(v_new[l]) || !aligned16(k_pools[l]) || !aligned16(v_pools[l]))
+            return DELTA_ERR_INVALID_ARG;
+        a.k_new[l] = static_cast<const uint4*>(k_new[l]);
+        a.v_new[l] = static_cast<const uint4*>(v_new[l]);
+        a.k_pool[l] = static_cast<uint4*>(k_pools[l]);
+        a.v_pool[l] = static_cast<uint4*>(v_pools[l]);
+    }
+    const int row_vecs = desc->head_dim * elem_bytes(desc->dtype) / 16;
+    return launch_pdl(kv_append_layers_kernel, dim3(pt->batch, desc->num_kv_heads, num_layers), dim3(32), 0,
+                      static_cast<cudaStream_t>(stream), a, pt->page_indptr, pt->page_indices, pt->kv_len,
+                      desc->num_kv_heads, row_vecs, desc->num_phys_pages);
 }
 
 delta_status delta_full_attn(const delta_desc* desc, const delta_page_table* pt, const void* q, const void* k_pool,

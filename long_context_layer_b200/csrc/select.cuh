@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     __shared__ uint32_t s_digit, s_above;
 
     const int b = blockIdx.x, tid = threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
     int n = p.kv_len[b];
     const int npg = p.indptr[b + 1] - p.indptr[b];
     if (n < 0) n = 0;
@@ -190,19 +192,21 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     if (tid == 0) p.sel_cnt[b] = min(total, p.sel_stride);
 }
 
-// ------------------------------------------------------------------ kv append kernel
-__global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
-                                 uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
-                                 const int32_t* __restrict__ indptr, const int32_t* __restrict__ indices,
-                                 const int32_t* __restrict__ kv_len, int Hkv, int row_vecs,
-                                 int64_t num_phys_pages) {
-    const int b = blockIdx.x, g = blockIdx.y;
+// ------------------------------------------------------------------ kv append kernels
+// Copy one token row (row_vecs 16-byte vectors) of KV head g of sequence b into slot
+// (kv_len-1) % 16 of logical page (kv_len-1) / 16.  Out-of-range pages are skipped (the attention
+// call that follows on the same page table flags them).
+__device__ __forceinline__ void append_row(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                           uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                           const int32_t* __restrict__ indptr, const int32_t* __restrict__ indices,
+                                           const int32_t* __restrict__ kv_len, int Hkv, int row_vecs,
+                                           int64_t num_phys_pages, int b, int g) {
     const int n = kv_len[b];
     if (n <= 0) return;
     const int pos = n - 1;
     const int lp = pos / kPage, slot = pos % kPage;
     const int pbeg = indptr[b], npg = indptr[b + 1] - pbeg;
-    if (lp >= npg) return;                       // flagged by the attention call
+    if (lp >= npg) return;
     const int64_t phys = indices[pbeg + lp];
     if (phys < 0 || phys >= num_phys_pages) return;
     const size_t src = (size_t(b) * Hkv + g) * row_vecs;
@@ -211,6 +215,36 @@ __global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* _
         k_pool[dst + i] = k_new[src + i];
         v_pool[dst + i] = v_new[src + i];
     }
+}
+
+__global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                 uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                 const int32_t* __restrict__ indptr, const int32_t* __restrict__ indices,
+                                 const int32_t* __restrict__ kv_len, int Hkv, int row_vecs,
+                                 int64_t num_phys_pages) {
+    pdl_wait();
+    pdl_trigger();
+    append_row(k_new, v_new, k_pool, v_pool, indptr, indices, kv_len, Hkv, row_vecs, num_phys_pages, blockIdx.x,
+               blockIdx.y);
+}
+
+constexpr int kMaxAppendLayers = 64;
+struct AppendLayers {
+    const uint4* k_new[kMaxAppendLayers];
+    const uint4* v_new[kMaxAppendLayers];
+    uint4* k_pool[kMaxAppendLayers];
+    uint4* v_pool[kMaxAppendLayers];
+};
+
+// Every layer of a decode step in one launch: grid (batch, KV heads, layers).
+__global__ void kv_append_layers_kernel(const __grid_constant__ AppendLayers a, const int32_t* __restrict__ indptr,
+                                        const int32_t* __restrict__ indices, const int32_t* __restrict__ kv_len,
+                                        int Hkv, int row_vecs, int64_t num_phys_pages) {
+    pdl_wait();
+    pdl_trigger();
+    const int l = blockIdx.z;
+    append_row(a.k_new[l], a.v_new[l], a.k_pool[l], a.v_pool[l], indptr, indices, kv_len, Hkv, row_vecs,
+               num_phys_pages, blockIdx.x, blockIdx.y);
 }
 
 }  // namespace delta

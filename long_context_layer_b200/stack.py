@@ -4,8 +4,8 @@ Layer schedule (DELTA: Dynamic Layer-Aware Token Attention, ai.info summary,
 "Methodology in Plain English"): layers before the first delta-layer run full
 attention; a delta-layer runs full attention and refreshes the page selection;
 every other layer runs sparse attention over the selection of the most recent
-delta-layer of the same decode step.  Every layer first appends the current
-token's k and v to its own paged pool (the cache is kept in full).
+delta-layer of the same decode step.  The step starts by appending the current
+token's k and v to every layer's paged pool in one launch (the cache is kept in full).
 
 The runner only sequences C-ABI calls on one CUDA stream; it can capture the
 whole step in a CUDA graph so one replay launches every kernel of the step.
@@ -69,15 +69,15 @@ class DeltaStack:
     # ------------------------------------------------------------------ one step
     def launches_per_step(self, append: bool = True) -> int:
         per = {FULL: 1, DELTA: 2, SPARSE: 1}
-        return sum(per[k] + (1 if append else 0) for k in self.kinds)
+        return sum(per[k] for k in self.kinds) + (1 if append else 0)
 
     def step(self, q, k_new, v_new, k_pools, v_pools, out, append: bool = True, stream: int | None = None):
         st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
         d, pt, ws, wb = self.desc, self.pt, self.workspace, self.ws_bytes
         cur = -1
+        if append:      # every layer's new token in one launch (layers do not read each other's pools)
+            N.kv_append_layers(d, pt, k_new, v_new, k_pools, v_pools, st)
         for l, kind in enumerate(self.kinds):
-            if append:
-                N.kv_append(d, pt, k_new[l], v_new[l], k_pools[l], v_pools[l], st)
             if kind == FULL:
                 N.full_attn(d, pt, q[l], k_pools[l], v_pools[l], out[l], ws, wb, st)
             elif kind == DELTA:

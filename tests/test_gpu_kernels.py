@@ -264,6 +264,26 @@ def test_kv_append_writes_exactly_one_slot(L, dtype, D):
     assert idx <= allowed
 
 
+def test_kv_append_layers_matches_per_layer_append(L):
+    cfg = make_cfg(5, 2, 128, "bf16", [33, 16, 1, 100], layers=3, delta=(0,), extra_pool=5)
+    a = device_case(cfg, prefill="append")
+    b = device_case(cfg, prefill="append")
+    desc, pt = make_desc(L, cfg, a), make_pt(L, a)
+    for l in range(3):
+        L.kv_append(desc, pt, a.k_new[l], a.v_new[l], a.k_pools[l], a.v_pools[l], stream())
+    pt_b = make_pt(L, b)
+    L.kv_append_layers(desc, pt_b, b.k_new, b.v_new, b.k_pools, b.v_pools, stream())
+    torch.cuda.synchronize()
+    for l in range(3):
+        for pa, pb in ((a.k_pools[l], b.k_pools[l]), (a.v_pools[l], b.v_pools[l])):
+            for bb, n in enumerate(cfg.context_list):
+                for g in range(2):
+                    phys = a.case.page_indices[a.case.page_indptr[bb] + (n - 1) // 16]
+                    assert torch.equal(pa[phys, g, (n - 1) % 16], pb[phys, g, (n - 1) % 16])
+                    assert torch.equal(pb[phys, g, (n - 1) % 16], b.k_new[l][bb, g] if pa is a.k_pools[l] else
+                                       b.v_new[l][bb, g])
+
+
 # ----------------------------------------------------------------- device-side checks
 def test_corrupt_page_id_is_flagged_not_trapped(L):
     cfg = make_cfg(4, 1, 64, "f32", [300])
