@@ -1,6 +1,8 @@
 """Build the in-tree shared libraries with nvcc for sm_100a.
 
-    python -m long_context_layer_b200.build
+    python long_context_layer_b200/build.py [--force]
+
+(Run it by path: importing the package loads the library this script builds.)
 
 Produces long_context_layer_b200/libdelta_attn.so (the C ABI of include/delta_attn.h) and
 synth/libsynth_fill.so (the device-side input generator used by tests and the benchmark).

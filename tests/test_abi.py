@@ -13,8 +13,8 @@ HEADER = os.path.join(ROOT, "include", "delta_attn.h")
 
 @pytest.fixture(scope="module")
 def L():
-    from long_context_layer_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import long_context_layer_b200 as lib
     return lib
 
