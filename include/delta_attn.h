@@ -143,6 +143,28 @@ delta_status delta_full_attn(const delta_desc* desc, const delta_page_table* pt,
                              const void* q, const void* k_pool, const void* v_pool, void* o,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* delta_full_attn without a workspace argument, for callers that cannot allocate device
+ * memory themselves: code that runs inside a CUDA graph being captured or replayed, a
+ * real-time loop that must never call cudaMalloc, or a host framework that owns every
+ * allocation and exposes no allocator to plug-ins.  The paper has no counterpart; it is a
+ * property of this library's interface.
+ *
+ * Same inputs, output and results as delta_full_attn.  Its scratch is a fixed 8 MiB array
+ * inside the library (static device memory: every GPU that loads the library keeps it until
+ * the process exits).  The call allocates and frees nothing.  Shapes whose
+ * delta_workspace_size() exceeds 8 MiB return DELTA_ERR_UNSUPPORTED.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ * - All calls share the one array and it keeps the last call's contents: each call clears
+ *   its counters first (cudaMemsetAsync on `stream`).  Calls whose kernels overlap on the
+ *   GPU (other streams, other threads) race on the array and give wrong results; serialise
+ *   them on one stream.
+ * - Device-side check flags land in the shared array and are not reported; use
+ *   delta_full_attn with a workspace to read them. */
+delta_status delta_full_attn_noalloc(const delta_desc* desc, const delta_page_table* pt,
+                                     const void* q, const void* k_pool, const void* v_pool, void* o,
+                                     void* stream);
+
 /* Delta-layer: the same output as delta_full_attn, plus the page selection of each
  * sequence.  Page score (HEAD_SUM): S[b][j] = sum over all query heads h and tokens
  * t of page j of the softmax probability p[h][t].  Selection: sink pages, recency

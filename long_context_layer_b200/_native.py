@@ -26,7 +26,8 @@ DELTA_HEAD_SUM, DELTA_HEAD_MAX = 0, 1
 EXPORTED = [
     "delta_workspace_size", "delta_workspace_init", "delta_sel_capacity", "delta_kv_append",
     "delta_kv_append_layers",
-    "delta_full_attn", "delta_select_attn", "delta_sparse_attn", "delta_read_device_error",
+    "delta_full_attn", "delta_full_attn_noalloc", "delta_select_attn", "delta_sparse_attn",
+    "delta_read_device_error",
     "delta_status_string",
 ]
 
@@ -65,6 +66,8 @@ lib.delta_kv_append_layers.argtypes = [_D, _PT, _i32, _vpp, _vpp, _vpp, _vpp, _v
 lib.delta_kv_append_layers.restype = _i32
 lib.delta_full_attn.argtypes = [_D, _PT, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.delta_full_attn.restype = _i32
+lib.delta_full_attn_noalloc.argtypes = [_D, _PT, _vp, _vp, _vp, _vp, _vp]
+lib.delta_full_attn_noalloc.restype = _i32
 lib.delta_select_attn.argtypes = [_D, _PT, _SP, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]
 lib.delta_select_attn.restype = _i32
 lib.delta_sparse_attn.argtypes = [_D, _PT, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -135,6 +138,13 @@ def full_attn(desc, pt, q, k_pool, v_pool, o, workspace, ws_bytes: int, stream: 
     s = lib.delta_full_attn(ctypes.byref(desc), ctypes.byref(pt), ptr(q), ptr(k_pool), ptr(v_pool), ptr(o),
                             ptr(workspace), ws_bytes, stream)
     return _check(s, "delta_full_attn") if check else s
+
+
+def full_attn_noalloc(desc, pt, q, k_pool, v_pool, o, stream: int = 0, check: bool = True) -> int:
+    """delta_full_attn with the library's own fixed scratch instead of a caller workspace."""
+    s = lib.delta_full_attn_noalloc(ctypes.byref(desc), ctypes.byref(pt), ptr(q), ptr(k_pool), ptr(v_pool), ptr(o),
+                                    stream)
+    return _check(s, "delta_full_attn_noalloc") if check else s
 
 
 def select_attn(desc, pt, sp, q, k_pool, v_pool, o, sel_cnt, sel_pages, sel_stride: int, page_scores,

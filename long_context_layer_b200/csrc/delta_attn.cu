@@ -528,6 +528,27 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
                       size_t(pt->max_pages_per_seq) * sizeof(uint32_t), st, sp2);
 }
 
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch of delta_full_attn_noalloc: a fixed array in the library's own device memory, so the
+// call needs no workspace from the caller.  Every GPU that loads the library holds it until the
+// process exits.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kStaticScratchBytes];
+
+// Device address of the scratch array on the current device, looked up once per device.  In
+// host code the array's name only stands for the symbol; the kernel must get this address.
+unsigned char* noalloc_scratch() {
+    static unsigned char* addr[64] = {nullptr};
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
+    if (addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return nullptr;
+        addr[dev] = static_cast<unsigned char*>(ptr);
+    }
+    return addr[dev];
+}
+
 }  // namespace delta
 
 using namespace delta;
@@ -604,6 +625,23 @@ delta_status delta_full_attn(const delta_desc* desc, const delta_page_table* pt,
                              const void* v_pool, void* o, void* workspace, size_t ws_bytes, void* stream) {
     return run_attention(kModeFull, desc, pt, nullptr, nullptr, nullptr, 0, q, k_pool, v_pool, o, nullptr, nullptr, 0,
                          nullptr, workspace, ws_bytes, stream);
+}
+
+delta_status delta_full_attn_noalloc(const delta_desc* desc, const delta_page_table* pt, const void* q,
+                                     const void* k_pool, const void* v_pool, void* o, void* stream) {
+    delta_status s = check_desc(desc);
+    if (s != DELTA_OK) return s;
+    s = check_pt(pt);
+    if (s != DELTA_OK) return s;
+    if (pt->batch == 0) return DELTA_OK;
+    const WsLayout L = ws_layout(desc, pt->batch, pt->max_pages_per_seq);
+    if (L.total > kStaticScratchBytes) return DELTA_ERR_UNSUPPORTED;   // shape needs more scratch than the array holds
+    unsigned char* ws = noalloc_scratch();
+    if (ws == nullptr) return DELTA_ERR_CUDA;
+    // the error word and the split-arrival tickets must start at zero; the rest is overwritten
+    if (cudaMemsetAsync(ws, 0, L.part_ml, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DELTA_ERR_CUDA;
+    return run_attention(kModeFull, desc, pt, nullptr, nullptr, nullptr, 0, q, k_pool, v_pool, o, nullptr, nullptr, 0,
+                         nullptr, ws, kStaticScratchBytes, stream);
 }
 
 delta_status delta_select_attn(const delta_desc* desc, const delta_page_table* pt, const delta_select_params* sp,
