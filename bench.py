@@ -41,10 +41,45 @@ def parse():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
+    ap.add_argument("--print-source-hash", action="store_true", help="print the kernel-source hash and exit")
     return ap.parse_args()
 
 
 # ---------------------------------------------------------------------------- helpers
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources of the library (identifies the kernels a profile was taken on)."""
+    import hashlib
+    d = os.path.join(ROOT, "long_context_layer_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the full-layer decode from the committed ncu summary of this
+    workload, or None when the kernels changed since that capture."""
+    path = os.path.join(ROOT, "profiles", f"decode_full_layer_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_sources_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -409,7 +444,7 @@ def run_ours(args):
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                          "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_kernel, 3),
-                         "traffic": None},
+                         "traffic": profiled_traffic(cfg.name)},
             "breakdown_us_per_call": breakdown,
             "e2e": {"value": round(us_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
@@ -427,6 +462,9 @@ def run_ours(args):
 
 def main():
     args = parse()
+    if args.print_source_hash:
+        print(kernel_source_hash())
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -185,10 +185,11 @@ struct WarpPages {
 };
 
 struct SeqExtent {
-    int n;      // tokens (clamped)
-    int N;      // pages
-    int pbeg;   // first entry of the sequence in page_indices
-    int count;  // items to attend: N, or the selection length
+    int n;                  // tokens (clamped)
+    int N;                  // pages
+    int pbeg;               // first entry of the sequence in page_indices
+    int count;              // items to attend: N, or the selection length
+    const int32_t* table;   // the sequence's page-table row staged in shared memory, or null
 };
 
 template <typename P>
@@ -204,7 +205,7 @@ __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int
         atomicOr(p.err, kErrSel);
         return;
     }
-    const int64_t x = p.indices[ex.pbeg + lp];
+    const int64_t x = ex.table != nullptr ? ex.table[lp] : p.indices[ex.pbeg + lp];
     if (x < 0 || x >= p.num_phys_pages) {
         atomicOr(p.err, kErrPage);
         return;
@@ -239,15 +240,14 @@ __device__ __forceinline__ void pages_get(const WarpPages& w, int k, int& lp, in
     ph = __shfl_sync(0xffffffffu, a ? w.ph_a : w.ph_b, k & 31);
 }
 
-// Tokens and item count of sequence b, validated against the page table (bad values clamped
-// and flagged).
+// Tokens and pages of sequence b, validated against the page table (bad values clamped and
+// flagged).  Reads only the page table and kv_len, which are inputs of the whole step.
 template <typename P>
 __device__ __forceinline__ SeqExtent seq_extent(const P& p, int b) {
     SeqExtent ex;
     int n = p.kv_len[b];
     ex.pbeg = p.indptr[b];
     const int npg = p.indptr[b + 1] - ex.pbeg;
-    const int scnt = (p.mode == kModeSparse) ? p.sel_cnt[b] : 0;
     if (n < 0) n = 0;
     if (n > npg * kPage || n > p.max_pages * kPage) {
         if (threadIdx.x == 0) atomicOr(p.err, kErrLen);
@@ -256,27 +256,23 @@ __device__ __forceinline__ SeqExtent seq_extent(const P& p, int b) {
     ex.n = n;
     ex.N = (n + kPage - 1) / kPage;
     ex.count = ex.N;
-    if (p.mode == kModeSparse) {
-        const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
-        ex.count = scnt;
-        if (scnt < 0 || scnt > cap) {
-            if (threadIdx.x == 0) atomicOr(p.err, kErrSel);
-            ex.count = min(max(scnt, 0), cap);
-        }
-    }
+    ex.table = nullptr;
     return ex;
 }
 
-// Epilogue shared by the decode kernels.
-//
-// mo [NPART][kMaxGroup][D] and mml [NPART][kMaxGroup][2] (shared memory) hold NPART partial
-// states (base-2 running max, sum of exponentials, unnormalised output) of the G query heads
-// of this CTA.  The C CTAs of a thread-block cluster cover C consecutive splits of one
-// (sequence, KV head): each reduces its NPART states to one, the cluster merges those through
-// distributed shared memory (every CTA finalises a 1/C slice of the G x D outputs), and
-//   - with one cluster per (sequence, KV head) the slice is the final output;
-//   - with nC > 1 clusters each writes a cluster partial to the workspace, and the last CTA to
-//     arrive (an atomic ticket; nobody waits) merges the nC partials into the output.
+// Sparse layers: the number of selected pages (an output of the delta-layer: read after the wait).
+template <typename P>
+__device__ __forceinline__ void seq_count(const P& p, int b, SeqExtent& ex) {
+    if (p.mode != kModeSparse) return;
+    const int scnt = p.sel_cnt[b];
+    const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
+    ex.count = scnt;
+    if (scnt < 0 || scnt > cap) {
+        if (threadIdx.x == 0) atomicOr(p.err, kErrSel);
+        ex.count = min(max(scnt, 0), cap);
+    }
+}
+
 // Floats of the dedicated receive area of the cluster merge (never aliased with pipeline stages,
 // so other CTAs of the cluster may push into it while this CTA is still streaming pages).
 template <int D>

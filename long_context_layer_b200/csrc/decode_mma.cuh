@@ -68,7 +68,10 @@ struct MmaSmem {
     static constexpr size_t kMain = kStages > kMerge ? kStages : kMerge;
     static constexpr size_t kBars = size_t(kWarps) * STAGES * sizeof(uint64_t);
     static constexpr size_t kRecv = size_t(recv_floats<D>()) * sizeof(float);
-    static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kRecv;
+    // the page-table row of the sequence, staged for sparse layers (deep variant only: the
+    // shallow one must keep two CTAs per SM)
+    static constexpr int kTable = STAGES >= 6 ? 4096 : 0;
+    static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kRecv + size_t(kTable) * 4;
 };
 
 template <int D, int G, int STAGES>
@@ -82,6 +85,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         smem_raw + ((1024 - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kMain);
     float* recv = reinterpret_cast<float*>(smem + S::kMain + S::kBars);
+    int32_t* table = reinterpret_cast<int32_t*>(smem + S::kMain + S::kBars + S::kRecv);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g4 = lane >> 2, t4 = lane & 3;
@@ -102,11 +106,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
     // so full and delta layers resolve their pages before waiting for the previous kernel; the
     // sparse layers' page list is the output of the delta-layer and is read after the wait.
-    SeqExtent ex;
+    SeqExtent ex = seq_extent(p, b);
     int i0 = 0, nk = 0;
     WarpPages pages;
     auto setup = [&]() {
-        ex = seq_extent(p, b);
+        seq_count(p, b, ex);
         i0 = split * p.items_per_split;
         const int i1 = min(i0 + p.items_per_split, ex.count);
         nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
@@ -125,6 +129,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
                 prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.v_pool) + off, kPage * D * 2);
             }
         }
+    } else if (S::kTable > 0 && ex.N <= S::kTable) {
+        // stage the page-table row so that, after the wait, a selected page costs one load
+        for (int j = threadIdx.x; j < ex.N; j += kThreads) table[j] = p.indices[ex.pbeg + j];
+        __syncthreads();
+        ex.table = table;
     }
     pdl_wait();      // q, the pools and the selection are written by earlier kernels
     pdl_trigger();

@@ -49,11 +49,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
     // so full and delta layers resolve their pages before waiting for the previous kernel; the
     // sparse layers' page list is the output of the delta-layer and is read after the wait.
-    SeqExtent ex;
+    SeqExtent ex = seq_extent(p, b);
     int i0 = 0, nk = 0;
     WarpPages pages;
     auto setup = [&]() {
-        ex = seq_extent(p, b);
+        seq_count(p, b, ex);
         i0 = split * p.items_per_split;
         const int i1 = min(i0 + p.items_per_split, ex.count);
         nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
