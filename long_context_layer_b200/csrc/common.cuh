@@ -17,6 +17,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxGroup = 8;
 constexpr int kMaxSelectPages = 32768;
 constexpr int kSelectThreads = 1024;
+constexpr int kMaxQHeadsSelect = 256;   // query heads a delta-layer selection supports
 constexpr int kMaxSplits = 512;   // the merge stages G*S*12 bytes of split weights in shared memory
 constexpr uint32_t kWaitLimit = 1u << 24;   // try_wait polls before a stage wait gives up
 

@@ -20,7 +20,7 @@
 //                         The split partials of a (sequence, KV head) are merged by whichever
 //                         of its CTAs arrives last (an atomic ticket; no CTA ever waits), which
 //                         writes o and, for delta-layers, each head's (max, sum-exp) pair.
-//   score_select_kernel   one CTA per sequence: page score = sum over heads of
+//   score_select_kernel   one thread-block cluster per sequence: page score = sum over heads of
 //                         2^(m_hp - M_h) l_hp / L_h, then an MSB-first 4x8-bit radix select of
 //                         the k-th largest candidate score with shared-memory histograms,
 //                         lower-index tie-break by a block prefix scan, union with sink and
@@ -47,7 +47,6 @@ namespace delta {
 // ------------------------------------------------------------------ host side
 constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB each for D = 128), 2 CTAs/SM
 constexpr int kMmaStagesDeep = 6;  // when the whole grid fits one CTA per SM: twice the pages in flight
-constexpr int kMaxQHeadsSelect = 256;
 
 struct WsLayout {
     size_t err, tickets, part_ml, part_o, page_ml, total;
@@ -141,7 +140,8 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
 
 WsLayout ws_layout(const delta_desc* d, int batch, int max_pages) {
     WsLayout w{};
-    const int S = plan_splits(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages).clusters;
+    // room for as many cluster partials as there are splits (fit_plan never exceeds that)
+    const int S = plan_splits(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages).splits();
     const size_t rows = size_t(batch) * d->num_q_heads;
     size_t off = 0;
     w.err = off;        off += align256(64);
@@ -323,21 +323,44 @@ int max_active_clusters(const void* func, size_t smem, int cluster) {
     return n;
 }
 
-// Shrink a split plan until all its clusters are resident in one wave (when possible).
-SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units) {
-    for (;;) {
+// Fit a split plan to the clusters that can be resident at once.  Among cluster sizes C <= the
+// plan's, pick the (C, clusters) pair with the most CTAs (C * clusters <= the plan's splits) whose
+// units * clusters all fit in one wave; ties go to the larger cluster (fewer cross-cluster
+// partials).  Long sequences thus keep ~one wave of CTAs even where large clusters do not pack
+// into the GPCs.
+SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) {
+    const int s = pl.splits();
+    // Clusters meet through the workspace only when each gets at least 256 pages: below that the
+    // cross-cluster merge costs more than the extra CTAs gain.
+    const int max_clusters = items / 256 > 1 ? items / 256 : 1;
+    SplitPlan best = pl;
+    int best_ctas = -1;
+    for (int c = pl.cluster; c >= 1; --c) {
+        SplitPlan cand = pl;
+        cand.cluster = c;
+        cand.clusters = s / c < max_clusters ? s / c : max_clusters;
+        if (cand.clusters < 1) continue;
+        cand.deep = pl.deep && int64_t(units) * c * cand.clusters <= device_sm_count();
         size_t smem = 0;
-        const void* fn = decode_ptr(dtype, D, G, pl.deep, &smem);
+        const void* fn = decode_ptr(dtype, D, G, cand.deep, &smem);
         if (fn == nullptr) return pl;
-        const int maxc = max_active_clusters(fn, smem, pl.cluster);
-        if (int64_t(units) * pl.clusters <= maxc) return pl;
-        if (pl.clusters > 1) {
-            pl.clusters = maxc / units > 1 ? maxc / units : 1;
-            continue;
+        const int maxc = max_active_clusters(fn, smem, c);
+        if (int64_t(units) * cand.clusters > maxc) {
+            cand.clusters = maxc / units;
+            if (cand.clusters < 1) continue;
         }
-        if (pl.cluster == 1) return pl;   // more units than resident clusters: several waves
-        pl.cluster = (pl.cluster + 1) / 2;
+        const int ctas = c * cand.clusters;
+        if (ctas > best_ctas) {
+            best = cand;
+            best_ctas = ctas;
+        }
     }
+    if (best_ctas < 0) {   // more units than resident clusters even at size 1: several waves
+        best.cluster = 1;
+        best.clusters = 1;
+        best.deep = false;
+    }
+    return best;
 }
 
 // Launch with programmatic dependent launch: the kernel may be scheduled while the previous
@@ -472,7 +495,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     int items = pt->max_pages_per_seq;
     if (mode == kModeSparse && sel_stride_in < items) items = sel_stride_in;
     const SplitPlan plan = fit_plan(plan_splits(d->dtype, D, pt->batch, Hkv, items), d->dtype, D, Hq / Hkv,
-                                    pt->batch * Hkv);
+                                    pt->batch * Hkv, items);
     const int S = plan.splits();
     unsigned char* base = static_cast<unsigned char*>(ws);
 
@@ -521,11 +544,30 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     sp2.sel_stride = sel_stride_out;
     sp2.page_scores = page_scores;
     sp2.err = prm.err;
-    static int configured[64] = {0};
-    if (!set_smem_once(score_select_kernel, size_t(kMaxSelectPages) * sizeof(uint32_t), configured))
-        return DELTA_ERR_CUDA;
-    return launch_pdl(score_select_kernel, dim3(pt->batch), dim3(kSelectThreads),
-                      size_t(pt->max_pages_per_seq) * sizeof(uint32_t), st, sp2);
+    // one cluster of C CTAs per sequence, about 16K page partials per CTA
+    const int maxp = pt->max_pages_per_seq;
+    int C = int((int64_t(Hq) * maxp + 16383) / 16384);
+    C = C < 1 ? 1 : (C > 16 ? 16 : C);
+    const int chunk = (maxp + C - 1) / C;
+    const SelectSmem SL{chunk, C, Hq};
+    const size_t smem_max = SelectSmem{kMaxSelectPages, 16, kMaxQHeadsSelect}.bytes();
+    if (!configure_kernel(reinterpret_cast<const void*>(score_select_kernel), smem_max)) return DELTA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, pt->batch);
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = SL.bytes();
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, score_select_kernel, sp2, chunk) != cudaSuccess) return DELTA_ERR_CUDA;
+    return launch_status();
 }
 
 // ------------------------------------------------------------------ allocation-free variant

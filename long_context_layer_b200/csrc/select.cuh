@@ -54,13 +54,49 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& 
     return res;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const SelectParams p) {
-    extern __shared__ uint32_t keys[];  // [max_pages]
-    __shared__ uint32_t hist[512];   // radix histogram; first reused for per-head totals
+// Shared-memory plan of the selection cluster (dynamic): keys of this CTA's pages, per-head
+// partial totals received from every CTA, double-buffered histograms received from every CTA.
+struct SelectSmem {
+    int chunk, C, Hq;
+    __host__ __device__ size_t keys() const { return 0; }
+    __host__ __device__ size_t mz() const { return (size_t(chunk) * 4 + 15) & ~size_t(15); }
+    __host__ __device__ size_t hist() const { return mz() + size_t(C) * Hq * 8; }
+    __host__ __device__ size_t counts() const { return hist() + size_t(2) * C * 256 * 4; }
+    __host__ __device__ size_t bytes() const { return counts() + size_t(C) * 8; }
+};
+
+// One thread-block cluster per sequence; CTA r of C owns pages [r*chunk, (r+1)*chunk).
+// 1. per-head totals over the page partials, M_h = max_j m_hj and Z_h = sum_j 2^(m_hj - M_h) l_hj
+//    (each CTA over its pages, exchanged through distributed shared memory);
+// 2. page scores S_j = sum_h 2^(m_hj - M_h) l_hj / Z_h -> order-preserving keys;
+// 3. MSB-first 4 x 8-bit radix select of the k-th largest candidate key (histograms summed over
+//    the cluster), candidates being the pages neither sink nor recency;
+// 4. ascending compaction of sink U recency U {key > T} U {the first (k - #greater) keys == T in
+//    page order} with cluster-wide offsets.
+// Every exchange pushes into the other CTAs' shared memory and is followed by one cluster barrier,
+// so no CTA reads remote memory after the last barrier.
+__global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const SelectParams p, int chunk) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = int(cluster.num_blocks()), rank = int(cluster.block_rank());
+    auto cluster_barrier = [&]() {
+        if (C > 1) cluster.sync();
+        else __syncthreads();
+    };
+    extern __shared__ __align__(16) unsigned char sm[];
+    const int Hq = p.num_q_heads;
+    const SelectSmem L{chunk, C, Hq};
+    uint32_t* keys = reinterpret_cast<uint32_t*>(sm + L.keys());
+    float2* recv_mz = reinterpret_cast<float2*>(sm + L.mz());        // [C][Hq]
+    uint32_t* recv_hist = reinterpret_cast<uint32_t*>(sm + L.hist());  // [2][C][256]
+    int2* recv_cnt = reinterpret_cast<int2*>(sm + L.counts());         // [C]
+    __shared__ float headM[kMaxQHeadsSelect], headZ[kMaxQHeadsSelect];
+    __shared__ uint32_t hist[256];
     __shared__ int warp_sums[33];
     __shared__ uint32_t s_digit, s_above;
 
-    const int b = blockIdx.x, tid = threadIdx.x;
+    const int b = blockIdx.y, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
     pdl_wait();
     pdl_trigger();
     int n = p.kv_len[b];
@@ -68,23 +104,31 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     if (n < 0) n = 0;
     if (n > npg * kPage) n = max(npg, 0) * kPage;   // flagged by the decode kernel
     const int N = min((n + kPage - 1) / kPage, p.max_pages);
-    const int Hq = p.num_q_heads;
-    const int sinkP = (min(p.sink_tokens, n) + kPage - 1) / kPage;
-    const int recStart = (p.recency_tokens > 0) ? max(n - p.recency_tokens, 0) / kPage : N;
+    const int j0 = min(rank * chunk, N), j1 = min(j0 + chunk, N);   // this CTA's pages
+    const int nloc = j1 - j0;
+    const int sinkP = min((min(p.sink_tokens, n) + kPage - 1) / kPage, N);
+    const int recStart = (p.recency_tokens > 0) ? min(max(n - p.recency_tokens, 0) / kPage, N) : N;
+    auto forced = [&](int j) { return j < sinkP || j >= recStart; };
+    const int ncand = max(recStart - sinkP, 0);
+    const int k = p.budget_pages;
+    const bool take_all = ncand <= k;
 
-    // 1. per-head totals over the page partials: M_h = max_j m_hj, Z_h = sum_j 2^(m_hj - M_h) l_hj
-    //    (one warp per head, lanes stride over pages with an online max/sum, then a warp merge)
-    float* headM = reinterpret_cast<float*>(hist);          // reuse: Hq <= 256 floats each
-    float* headZ = headM + 256;
-    const int warp = tid >> 5, lane = tid & 31;
+    // 1. per-head partial totals over this CTA's pages (a warp per head), pushed to every CTA
     for (int h = warp; h < Hq; h += kSelectThreads / 32) {
         const float2* pm = p.page_ml + (size_t(b) * Hq + h) * p.max_pages;
         float M = -INFINITY, Z = 0.f;
-        for (int j = lane; j < N; j += 32) {
-            const float2 ml = pm[j];
-            const float Mn = fmaxf(M, ml.x);
-            Z = Z * exp2_approx(M - Mn) + ml.y * exp2_approx(ml.x - Mn);
-            M = Mn;
+        // four independent loads in flight per lane, then an online (max, sum) update
+        for (int j = j0 + lane; j < j1; j += 128) {
+            float2 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = (j + 32 * u < j1) ? pm[j + 32 * u] : make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float Mn = fmaxf(M, v[u].x);
+                const float mu = (Mn == -INFINITY) ? 0.f : Mn;
+                Z = Z * exp2_approx(M - mu) + v[u].y * exp2_approx(v[u].x - mu);
+                M = Mn;
+            }
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
@@ -94,40 +138,66 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
             Z = Z * exp2_approx(M - mu) + Zo * exp2_approx(Mo - mu);
             M = Mn;
         }
-        if (lane == 0) { headM[h] = M; headZ[h] = Z; }
+        if (lane < C) cluster.map_shared_rank(recv_mz, lane)[rank * Hq + h] = make_float2(M, Z);
+    }
+    cluster_barrier();
+    for (int h = tid; h < Hq; h += kSelectThreads) {
+        float M = -INFINITY, Z = 0.f;
+        for (int j = 0; j < C; ++j) {
+            const float2 v = recv_mz[j * Hq + h];
+            const float Mn = fmaxf(M, v.x);
+            const float mu = (Mn == -INFINITY) ? 0.f : Mn;
+            Z = Z * exp2_approx(M - mu) + v.y * exp2_approx(v.x - mu);
+            M = Mn;
+        }
+        headM[h] = M;
+        headZ[h] = Z;
     }
     __syncthreads();
-    // 2. page scores S_j = sum_h 2^(m_hj - M_h) * l_hj / Z_h
-    for (int j = tid; j < N; j += kSelectThreads) {
+
+    // 2. page scores of this CTA's pages
+    for (int j = j0 + tid; j < j1; j += kSelectThreads) {
         float sc = 0.f;
-        for (int h = 0; h < Hq; ++h) {
-            const float2 ml = p.page_ml[(size_t(b) * Hq + h) * p.max_pages + j];
+        const float2* pm = p.page_ml + size_t(b) * Hq * p.max_pages + j;
+        int h = 0;
+        for (; h + 8 <= Hq; h += 8) {   // eight independent loads in flight
+            float2 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = pm[size_t(h + u) * p.max_pages];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sc += exp2_approx(v[u].x - headM[h + u]) * v[u].y / headZ[h + u];
+        }
+        for (; h < Hq; ++h) {
+            const float2 ml = pm[size_t(h) * p.max_pages];
             sc += exp2_approx(ml.x - headM[h]) * ml.y / headZ[h];
         }
-        keys[j] = order_key(sc);
+        keys[j - j0] = order_key(sc);
         if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
     }
     __syncthreads();
 
-    auto forced = [&](int j) { return j < sinkP || j >= recStart; };
-    // 2. number of candidates (pages neither sink nor recency)
-    int my_c = 0;
-    for (int j = tid; j < N; j += kSelectThreads) my_c += forced(j) ? 0 : 1;
-    int ncand;
-    block_exclusive_scan(my_c, warp_sums, ncand);
-    const int k = p.budget_pages;
-
-    // 3. radix select of the k-th largest candidate key (only when candidates exceed k)
+    // 3. radix select of the k-th largest candidate key over the whole cluster
     uint32_t T = 0, need_eq = 0;
-    bool take_all = ncand <= k;
     if (!take_all && k > 0) {
         uint32_t prefix = 0, mask = 0, kk = k;
-        for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int pass = 0, shift = 24; shift >= 0; ++pass, shift -= 8) {
             for (int i = tid; i < 256; i += kSelectThreads) hist[i] = 0;
             __syncthreads();
-            for (int j = tid; j < N; j += kSelectThreads) {
-                const uint32_t key = keys[j];
+            for (int j = j0 + tid; j < j1; j += kSelectThreads) {
+                const uint32_t key = keys[j - j0];
                 if (!forced(j) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            uint32_t* rh = recv_hist + (pass & 1) * C * 256;
+            for (int i = tid; i < C * 256; i += kSelectThreads) {
+                const int j = i >> 8, bin = i & 255;
+                cluster.map_shared_rank(rh, j)[rank * 256 + bin] = hist[bin];
+            }
+            cluster_barrier();
+            if (tid < 256) {
+                uint32_t t = 0;
+                for (int j = 0; j < C; ++j) t += rh[j * 256 + tid];
+                hist[tid] = t;
             }
             __syncthreads();
             if (tid < 32) {
@@ -158,30 +228,50 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
             __syncthreads();
         }
         T = prefix;
-        need_eq = kk;  // how many of the keys equal to T are taken (lowest page indices first)
+        need_eq = kk;   // how many of the keys equal to T are taken (lowest page indices first)
     }
 
-    // 4. rank of each T-valued candidate among equals, then the ascending compaction
-    const int chunk = (N + kSelectThreads - 1) / kSelectThreads;
-    const int jb = tid * chunk, je = min(jb + chunk, N);
-    int eq_cnt = 0;
-    if (!take_all && k > 0)
-        for (int j = jb; j < je; ++j) eq_cnt += (!forced(j) && keys[j] == T) ? 1 : 0;
-    int eq_tot;
-    int eq_rank = block_exclusive_scan(eq_cnt, warp_sums, eq_tot);
+    // 4. cluster-wide offsets, then the ascending compaction of this CTA's pages
+    const int per = (nloc + kSelectThreads - 1) / kSelectThreads;
+    const int jb = j0 + tid * per, je = min(jb + per, j1);
+    const bool radix = !take_all && k > 0;
+    int eq_cnt = 0, gtf_cnt = 0;
+    for (int j = jb; j < je; ++j) {
+        if (forced(j)) { ++gtf_cnt; continue; }
+        if (take_all) { ++gtf_cnt; continue; }
+        if (!radix) continue;
+        const uint32_t key = keys[j - j0];
+        if (key > T) ++gtf_cnt;
+        else if (key == T) ++eq_cnt;
+    }
+    int eq_tot_loc, gtf_tot_loc;
+    const int eq_rank_loc = block_exclusive_scan(eq_cnt, warp_sums, eq_tot_loc);
+    block_exclusive_scan(gtf_cnt, warp_sums, gtf_tot_loc);
+    if (tid < C) cluster.map_shared_rank(recv_cnt, tid)[rank] = make_int2(eq_tot_loc, gtf_tot_loc);
+    cluster_barrier();
+    int eq_cum = 0, eq_before = 0, sel_before = 0, total = 0;
+    for (int j = 0; j < C; ++j) {
+        const int2 v = recv_cnt[j];
+        const int taken = min(max(int(need_eq) - eq_cum, 0), v.x);   // T-valued pages of CTA j that are kept
+        if (j < rank) {
+            sel_before += v.y + taken;
+            eq_before += v.x;
+        }
+        total += v.y + taken;
+        eq_cum += v.x;
+    }
     auto selected = [&](int j, int& eq_seen) -> bool {
-        if (forced(j)) return true;
-        if (take_all) return true;
-        if (k <= 0) return false;
-        const uint32_t key = keys[j];
+        if (forced(j) || take_all) return true;
+        if (!radix) return false;
+        const uint32_t key = keys[j - j0];
         if (key > T) return true;
-        if (key == T) return (uint32_t)(eq_rank + eq_seen++) < need_eq;
+        if (key == T) return uint32_t(eq_before + eq_rank_loc + eq_seen++) < need_eq;
         return false;
     };
     int cnt = 0, seen = 0;
     for (int j = jb; j < je; ++j) cnt += selected(j, seen) ? 1 : 0;
-    int total;
-    int pos = block_exclusive_scan(cnt, warp_sums, total);
+    int local_total;
+    int pos = sel_before + block_exclusive_scan(cnt, warp_sums, local_total);
     seen = 0;
     for (int j = jb; j < je; ++j) {
         if (selected(j, seen)) {
@@ -189,7 +279,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
             ++pos;
         }
     }
-    if (tid == 0) p.sel_cnt[b] = min(total, p.sel_stride);
+    if (rank == 0 && tid == 0) p.sel_cnt[b] = min(total, p.sel_stride);
 }
 
 // ------------------------------------------------------------------ kv append kernels

@@ -185,6 +185,37 @@ def test_select_attn_matches_oracle(L, G, Hkv, D, dtype, ctx, k, sink, rec, plan
         assert ok, f"b={b}: gpu {gsel} vs oracle {ref_sel}"
 
 
+def test_select_exact_ties_across_cluster_ctas(L):
+    # Identical keys give identical page scores: the selection must take the lowest-index
+    # candidates, and with 32 query heads x 1025 pages the selection runs as a 3-CTA cluster
+    # whose chunk boundaries fall inside the selected range.
+    n, k = 16384 + 5, 700
+    cfg = make_cfg(8, 4, 128, "bf16", [n], budget_pages=k, sink=16, rec=256)
+    dc = device_case(cfg)
+    dc.k_pools[0].fill_(1.0)
+    desc, pt = make_desc(L, cfg, dc), make_pt(L, dc)
+    ws, nb = workspace(L, desc, dc)
+    sp = L.DeltaSelectParams(k, 16, 256, L.DELTA_HEAD_SUM)
+    stride = L.sel_capacity(sp)
+    maxp = dc.case.max_pages_per_seq
+    assert 32 * maxp > 2 * 16384
+    sel_cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sel_pages = torch.full((1, stride), -1, dtype=torch.int32, device="cuda")
+    scores = torch.zeros((1, maxp), dtype=torch.float32, device="cuda")
+    L.select_attn(desc, pt, sp, dc.q[0], dc.k_pools[0], dc.v_pools[0], dc.out[0], sel_cnt, sel_pages, stride,
+                  scores, ws, nb, stream())
+    ok_flags(L, ws)
+    K = np.ones((4, n, 128))
+    V = oracle_kv(dc.case, 0, 0)[1]
+    ref, p = O.full_attention(dc.case.q(0)[0].astype(np.float64), K, V)
+    assert_close(dc.out[0].float().cpu().numpy()[0], ref, "bf16", "o")
+    S = O.page_scores(p, 16)
+    np.testing.assert_allclose(scores.cpu().numpy()[0, :len(S)], S, rtol=2e-5)
+    got = sel_pages.cpu().numpy()[0, :int(sel_cnt.item())].tolist()
+    assert got == O.select_pages(S, n, 16, k, 16, 256)
+    assert got[:k + 1] == list(range(k + 1))
+
+
 # ----------------------------------------------------------------- sparse attention
 @pytest.mark.parametrize("G,Hkv,D,dtype,ctx", [
     (8, 1, 64, "f32", [1024]), (7, 4, 128, "bf16", [8192, 333]), (5, 2, 128, "bf16", [1000]),
