@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
     ap.add_argument("--print-source-hash", action="store_true", help="print the kernel-source hash and exit")
+    ap.add_argument("--drift-checks", type=int, default=10, help="oracle selection checks along a trajectory")
     return ap.parse_args()
 
 
@@ -297,6 +298,89 @@ def run_reference(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------- drifting trajectory
+def run_trajectory(args, cfg):
+    """The drifting workload: one CUDA graph per decode step replayed along the trajectory, the
+    cache growing one token per step and the planted keys moving every `drift_every` steps.
+    Reports per-step latency and, on sampled steps, the rate at which the GPU selection of
+    sequence 0 at the first delta-layer matches the fp64 oracle's."""
+    import numpy as np
+    import torch
+    from long_context_layer_b200.stack import DeltaStack
+    from synth.trajectory import Trajectory
+
+    dist, rank, world, local = dist_init()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    tr = Trajectory(cfg, device=device)
+    dc = tr.dc
+    stack = DeltaStack(cfg.layer_kinds(), cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr,
+                       dc.indices, dc.kv_len, tr.case0.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages,
+                       cfg.sink_tokens, cfg.recency_tokens)
+    tr.prepare(0)
+    g = stack.capture(dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+    flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    steps = min(args.steps, cfg.steps)
+    check_every = max(steps // max(args.drift_checks, 1), 1)
+    checks = set(range(0, steps, check_every)) if args.drift_checks > 0 else set()
+    lat, matched, checked = [], 0, 0
+    ld = cfg.layer_kinds().index("delta")
+    for step in range(steps):
+        tr.prepare(step)
+        for _ in range(args.warmup if step == 0 else 0):
+            g.replay()
+        flush.fill_(1)
+        flush_rd.sum()
+        barrier(dist, device)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        g.replay()
+        s1.record(stream)
+        s1.synchronize()
+        lat.append(s0.elapsed_time(s1) * 1000.0)
+        if rank == 0 and step in checks:
+            from oracle import delta_oracle as O
+            from synth import rng
+            case = tr.case_at(step)
+            n = int(case.n[0])
+            K = np.stack([case.kv_logical(rng.T_K, ld, 0, h) for h in range(cfg.num_kv_heads)]).astype(np.float64)
+            V = np.stack([case.kv_logical(rng.T_V, ld, 0, h) for h in range(cfg.num_kv_heads)]).astype(np.float64)
+            _, p = O.full_attention(case.q(ld)[0].astype(np.float64), K, V)
+            ref = O.select_pages(O.page_scores(p, cfg.page_size), n, cfg.page_size, cfg.budget_pages,
+                                 cfg.sink_tokens, cfg.recency_tokens)
+            matched += int(stack.selection(stack.delta_layers.index(ld))[0] == ref)
+            checked += 1
+    per = np.array(lat)
+    us = max_over_ranks(dist, float(per.mean()), device)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": round(us / 1000, 6), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "layers": cfg.num_layers, "delta_layers": list(cfg.delta_layers),
+                       "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
+                       "batch": cfg.batch, "start_context": int(tr.case0.n.max()), "drift_every": cfg.drift_every,
+                       "drift_shift": cfg.drift_shift, "budget_tokens": cfg.budget_tokens,
+                       "l2": "flushed before every timed replay (2xL2 write, then 2xL2 read)"},
+            "trajectory": {"per_step_us": {"mean": round(float(per.mean()), 3),
+                                           "median": round(float(np.median(per)), 3),
+                                           "p99": round(float(np.percentile(per, 99)), 3),
+                                           "first": round(float(per[0]), 3), "last": round(float(per[-1]), 3)},
+                           "selection_match_rate": (round(matched / checked, 4) if checked else None),
+                           "selection_checks": checked,
+                           "selection_check": "sequence 0, first delta-layer, exact match with the fp64 oracle"},
+            "gpu_launches": stack.launches_per_step() * steps,
+        }
+        print(json.dumps(line), flush=True)
+    del g
+    stack.graph = None
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -467,6 +551,11 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args)
+        return
+    from synth import configs as C
+    cfg = C.CONFIGS[args.config]
+    if cfg.steps > 1:
+        run_trajectory(args, cfg)
     else:
         run_ours(args)
 

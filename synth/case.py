@@ -30,6 +30,7 @@ class Case:
         self.key = rng.stream_key(cfg.seed, cfg.cfg_id)
         P = cfg.page_size
         self.n = np.array(cfg.contexts(step), dtype=np.int64)            # tokens attended per sequence
+        self.n0 = np.array(cfg.contexts(0), dtype=np.int64)              # at the first step of the trajectory
         # Pages are allocated for the longest context the trajectory reaches.
         self.n_max_traj = np.array(cfg.contexts(cfg.steps - 1), dtype=np.int64)
         pages_needed = -(-self.n_max_traj // P)
@@ -81,12 +82,13 @@ class Case:
             return self._plant_cache[ck]
         c = self.cfg
         lo = c.sink_tokens
+        n0 = int(self.n0[b])                       # planted positions are drawn once, at the first step
         if c.drift_every:
             # every shifted block must stay inside the prefilled zone
-            hi = int(self.n[b]) - 1 - c.recency_tokens - c.drift_shift * ((c.steps - 1) // c.drift_every)
+            hi = n0 - 1 - c.recency_tokens - c.drift_shift * ((c.steps - 1) // c.drift_every)
         else:
-            hi = int(self.n[b]) - c.recency_tokens
-        hi = min(hi, int(self.n[b]) - 1)          # the current token is never planted
+            hi = n0 - c.recency_tokens
+        hi = min(hi, n0 - 1)                       # the current token is never planted
         count = min(c.planted, max(hi - lo, 0))   # short contexts plant fewer keys
         if count == 0:
             out = np.zeros(0, dtype=np.int64)

@@ -48,7 +48,42 @@ __global__ void fill_kernel(void* pool, int is_bf16, int64_t num_phys_pages, int
     }
 }
 
+// out[l][b][g][d] = generator value of (tensor, l, b, g, pos[b], d) for layers 0..L-1: the token
+// each sequence appends at this decode step.
+__global__ void fill_tokens_kernel(void* out, int is_bf16, int Hkv, int D, const int32_t* __restrict__ pos,
+                                   uint64_t key, int tensor, float scale) {
+    const int l = blockIdx.x, b = blockIdx.y, B = gridDim.y;
+    const int p = pos[b];
+    for (int e = threadIdx.x; e < Hkv * D; e += blockDim.x) {
+        const int g = e / D, d = e % D;
+        const uint64_t hi = ((((uint64_t(tensor) << 6) | uint64_t(l)) << 6 | uint64_t(b)) << 6 | uint64_t(g)) << 28;
+        const uint64_t c = hi | (uint64_t(p) << 8) | uint64_t(d);
+        const uint64_t r = mix64(key + (c + 1ull) * 0x9E3779B97F4A7C15ull);
+        const int64_t s = int64_t(r & 0xFFFF) + int64_t((r >> 16) & 0xFFFF) + int64_t((r >> 32) & 0xFFFF) +
+                          int64_t(r >> 48);
+        const float x = __fmul_rn(float(s - 131070), scale);
+        const size_t o = ((size_t(l) * B + b) * Hkv + g) * D + d;
+        if (is_bf16) {
+            uint32_t u = __float_as_uint(x);
+            u = u + 0x7FFFu + ((u >> 16) & 1u);
+            reinterpret_cast<uint16_t*>(out)[o] = uint16_t(u >> 16);
+        } else {
+            reinterpret_cast<float*>(out)[o] = x;
+        }
+    }
+}
+
 }  // namespace
+
+extern "C" int synth_fill_tokens(void* out, int is_bf16, int L, int B, int Hkv, int D, const int32_t* pos,
+                                 uint64_t key, int tensor, float scale, void* stream) {
+    if (out == nullptr || pos == nullptr || L <= 0 || L > 64 || B <= 0 || B > 64 || Hkv <= 0 || Hkv > 64 || D <= 0 ||
+        D > 256 || tensor < 0 || tensor > 3)
+        return 1;
+    fill_tokens_kernel<<<dim3(L, B), 256, 0, static_cast<cudaStream_t>(stream)>>>(out, is_bf16, Hkv, D, pos, key,
+                                                                                  tensor, scale);
+    return cudaPeekAtLastError() == cudaSuccess ? 0 : 2;
+}
 
 extern "C" int synth_fill_kv(void* pool, int is_bf16, int64_t num_phys_pages, int Hkv, int D,
                              const int32_t* indptr, const int32_t* indices, const int32_t* fill_len,

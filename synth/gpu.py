@@ -29,6 +29,10 @@ def fill_lib():
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_uint64, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p]
         lib.synth_fill_kv.restype = ctypes.c_int
+        lib.synth_fill_tokens.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int, ctypes.c_float,
+                                          ctypes.c_void_p]
+        lib.synth_fill_tokens.restype = ctypes.c_int
         _LIB = lib
     return _LIB
 
@@ -118,6 +122,42 @@ class DeviceCase:
         dev = self.device
         pool[torch.from_numpy(p.astype(np.int64)).to(dev), torch.from_numpy(g.astype(np.int64)).to(dev),
              torch.from_numpy(s.astype(np.int64)).to(dev)] = to_device(rows, self.dtype, dev)
+
+    def fill_new_tokens(self, pos: torch.Tensor) -> None:
+        """k_new / v_new of every layer <- generator values at positions pos[b] (device int32)."""
+        c = self.cfg
+        assert self.layers == list(range(len(self.layers)))
+        st = torch.cuda.current_stream(self.device).cuda_stream
+        for tensor, buf in ((rng.T_K, self.k_new), (rng.T_V, self.v_new)):
+            r = fill_lib().synth_fill_tokens(buf.data_ptr(), 1 if c.dtype == "bf16" else 0, len(self.layers), c.batch,
+                                             c.num_kv_heads, c.head_dim, pos.data_ptr(), self.case.key, tensor,
+                                             float(rng.NORMAL_SCALE), st)
+            if r != 0:
+                raise RuntimeError(f"synth_fill_tokens failed ({r})")
+
+    def replant(self, step: int) -> None:
+        """Drift: move every layer's planted keys to their positions at `step` (the previous
+        positions get their generator values back)."""
+        c, case = self.cfg, self.case
+        if c.planted == 0 or not c.drift_every:
+            return
+        prev_step = max(step - c.drift_every, 0)
+        dev = self.device
+        for li, l in enumerate(self.layers):
+            P, G, S, R = [], [], [], []
+            for b in range(c.batch):
+                for g in range(c.num_kv_heads):
+                    old = case.planted_positions(l, b, g, prev_step)
+                    P.append(case.page_indices[case.page_indptr[b] + old // 16])
+                    G.append(np.full(old.size, g))
+                    S.append(old % 16)
+                    R.append(case.kv_base(rng.T_K, l, b, g, old))
+            dev_idx = lambda a: torch.from_numpy(np.concatenate(a).astype(np.int64)).to(dev)
+            # restore first, then plant (two scatters: an old and a new position may coincide)
+            self.k_pools[li][dev_idx(P), dev_idx(G), dev_idx(S)] = to_device(np.concatenate(R), self.dtype, dev)
+            p, g, s_, rows = self.planted_index(l, step)
+            self.k_pools[li][torch.from_numpy(p.astype(np.int64)).to(dev), torch.from_numpy(g.astype(np.int64)).to(dev),
+                             torch.from_numpy(s_.astype(np.int64)).to(dev)] = to_device(rows, self.dtype, dev)
 
     def pool_row(self, layer_idx: int, tensor: int, b: int, g: int, pos: int) -> torch.Tensor:
         c = self.case
