@@ -71,8 +71,10 @@ typedef enum { DELTA_F32 = 0, DELTA_BF16 = 1 } delta_dtype;
 
 /* How per-token attention is aggregated over query heads for the page score. */
 typedef enum {
-    DELTA_HEAD_SUM = 0,  /* softmax probability summed over all query heads (implemented) */
-    DELTA_HEAD_MAX = 1   /* maximum over heads, the page's own wording (not implemented: UNSUPPORTED) */
+    DELTA_HEAD_SUM = 0,  /* S_j = sum over query heads h and tokens t of page j of p[h][t] */
+    DELTA_HEAD_MAX = 1   /* S_j = sum over tokens t of page j of max_h p[h][t] ("for each token they take
+                            the maximum attention weight across heads", ai.info summary, "Methodology in
+                            Plain English"); needs delta_workspace_size_reduce(..., DELTA_HEAD_MAX) */
 } delta_head_reduce;
 
 /* Shape of one attention layer.  Supported: head_dim 64 or 128, page_size 16,
@@ -112,6 +114,12 @@ typedef struct {
  * device.  The workspace is scratch owned by the caller; it must be 256-byte
  * aligned and zero-filled once (delta_workspace_init) before first use. */
 size_t delta_workspace_size(const delta_desc* desc, int32_t batch, int32_t max_pages_per_seq);
+
+/* Workspace for delta_select_attn with the given head reduction: DELTA_HEAD_MAX also keeps
+ * every query head's per-token logits (batch * num_q_heads * max_pages_per_seq * 16 floats);
+ * DELTA_HEAD_SUM needs exactly delta_workspace_size().  0 for an invalid reduce. */
+size_t delta_workspace_size_reduce(const delta_desc* desc, int32_t batch, int32_t max_pages_per_seq,
+                                   int32_t reduce);
 
 /* Zero-fill a workspace (enqueued on `stream`). */
 delta_status delta_workspace_init(void* workspace, size_t ws_bytes, void* stream);
@@ -167,7 +175,8 @@ delta_status delta_full_attn_noalloc(const delta_desc* desc, const delta_page_ta
 
 /* Delta-layer: the same output as delta_full_attn, plus the page selection of each
  * sequence.  Page score (HEAD_SUM): S[b][j] = sum over all query heads h and tokens
- * t of page j of the softmax probability p[h][t].  Selection: sink pages, recency
+ * t of page j of the softmax probability p[h][t]; (HEAD_MAX) the sum over the page's
+ * tokens of the maximum over heads of p[h][t].  Selection: sink pages, recency
  * pages and the budget_pages best remaining pages, written ascending to
  * sel_pages[b][0..sel_cnt[b]).  page_scores may be NULL; when given, S is written
  * for j < ceil(kv_len[b]/page_size).  sel_stride must be >= delta_sel_capacity().

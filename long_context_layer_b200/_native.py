@@ -24,7 +24,7 @@ DELTA_F32, DELTA_BF16 = 0, 1
 DELTA_HEAD_SUM, DELTA_HEAD_MAX = 0, 1
 
 EXPORTED = [
-    "delta_workspace_size", "delta_workspace_init", "delta_sel_capacity", "delta_kv_append",
+    "delta_workspace_size", "delta_workspace_size_reduce", "delta_workspace_init", "delta_sel_capacity", "delta_kv_append",
     "delta_kv_append_layers",
     "delta_full_attn", "delta_full_attn_noalloc", "delta_select_attn", "delta_sparse_attn",
     "delta_read_device_error",
@@ -55,6 +55,8 @@ _D, _PT, _SP = ctypes.POINTER(DeltaDesc), ctypes.POINTER(DeltaPageTable), ctypes
 
 lib.delta_workspace_size.argtypes = [_D, _i32, _i32]
 lib.delta_workspace_size.restype = _sz
+lib.delta_workspace_size_reduce.argtypes = [_D, _i32, _i32, _i32]
+lib.delta_workspace_size_reduce.restype = _sz
 lib.delta_workspace_init.argtypes = [_vp, _sz, _vp]
 lib.delta_workspace_init.restype = _i32
 lib.delta_sel_capacity.argtypes = [_SP, _i32]
@@ -105,6 +107,10 @@ def _check(status: int, where: str) -> int:
 
 def workspace_size(desc: DeltaDesc, batch: int, max_pages_per_seq: int) -> int:
     return lib.delta_workspace_size(ctypes.byref(desc), batch, max_pages_per_seq)
+
+
+def workspace_size_reduce(desc: DeltaDesc, batch: int, max_pages_per_seq: int, reduce: int) -> int:
+    return lib.delta_workspace_size_reduce(ctypes.byref(desc), batch, max_pages_per_seq, reduce)
 
 
 def workspace_init(workspace, nbytes: int, stream: int = 0) -> None:

@@ -163,6 +163,7 @@ struct DecodeParams {
     float2* page_ml;  // [B][Hq][max_pages] per-page (max, sum) for delta-layers
     void* o;          // [B][Hq][D] output
     int32_t num_clusters;   // clusters along the split dimension (num_splits = cluster size * this)
+    float* logits;          // [B][Hq][max_pages*16] base-2 logits (delta-layers in HEAD_MAX mode), else null
     int* tickets;     // [B][Hkv] arrival counters of the split CTAs, zero between launches
     int* err;
 };

@@ -213,6 +213,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     };
     // Delta-layers: page partials from the unrounded probabilities (max logit, sum of 2^(s - max))
     auto page_partials = [&](const float (&sc)[4], int lp) {
+        if (p.logits != nullptr) {
+            // per-token logits of this page (HEAD_MAX scoring): tokens g4, g4+8; heads 2*t4, 2*t4+1
+            float* lg = p.logits + (size_t(b) * Hq + h0) * (size_t(p.max_pages) * kPage) + size_t(lp) * kPage;
+            const size_t hs = size_t(p.max_pages) * kPage;
+            if (2 * t4 < G) { lg[2 * t4 * hs + g4] = sc[0]; lg[2 * t4 * hs + g4 + 8] = sc[2]; }
+            if (2 * t4 + 1 < G) { lg[(2 * t4 + 1) * hs + g4] = sc[1]; lg[(2 * t4 + 1) * hs + g4 + 8] = sc[3]; }
+        }
         float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {

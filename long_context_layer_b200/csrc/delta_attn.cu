@@ -49,7 +49,7 @@ constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB 
 constexpr int kMmaStagesDeep = 6;  // when the whole grid fits one CTA per SM: twice the pages in flight
 
 struct WsLayout {
-    size_t err, tickets, part_ml, part_o, page_ml, total;
+    size_t err, tickets, part_ml, part_o, page_ml, logits, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -138,7 +138,8 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
     return pl;
 }
 
-WsLayout ws_layout(const delta_desc* d, int batch, int max_pages) {
+// with_logits: room for per-token logits of every query head (delta-layers scoring with HEAD_MAX)
+WsLayout ws_layout(const delta_desc* d, int batch, int max_pages, bool with_logits = false) {
     WsLayout w{};
     // room for as many cluster partials as there are splits (fit_plan never exceeds that)
     const int S = plan_splits(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages).splits();
@@ -149,6 +150,7 @@ WsLayout ws_layout(const delta_desc* d, int batch, int max_pages) {
     w.part_ml = off;    off += align256(rows * S * sizeof(float2));
     w.part_o = off;     off += align256(rows * S * d->head_dim * sizeof(float));
     w.page_ml = off;    off += align256(rows * size_t(max_pages) * sizeof(float2));
+    w.logits = off;     off += with_logits ? align256(rows * size_t(max_pages) * kPage * sizeof(float)) : 0;
     w.total = off;
     return w;
 }
@@ -473,7 +475,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     if (mode == kModeDelta) {
         if (sp == nullptr) return DELTA_ERR_INVALID_ARG;
         if (sp->budget_pages < 0 || sp->sink_tokens < 0 || sp->recency_tokens < 0) return DELTA_ERR_INVALID_ARG;
-        if (sp->reduce != DELTA_HEAD_SUM) return sp->reduce == DELTA_HEAD_MAX ? DELTA_ERR_UNSUPPORTED : DELTA_ERR_INVALID_ARG;
+        if (sp->reduce != DELTA_HEAD_SUM && sp->reduce != DELTA_HEAD_MAX) return DELTA_ERR_INVALID_ARG;
         if (d->num_q_heads > kMaxQHeadsSelect) return DELTA_ERR_UNSUPPORTED;
     }
     if (pt->batch == 0) return DELTA_OK;
@@ -488,7 +490,8 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
         if (sel_cnt_in == nullptr || sel_pages_in == nullptr || sel_stride_in <= 0) return DELTA_ERR_INVALID_ARG;
     }
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DELTA_ERR_WORKSPACE;
-    const WsLayout L = ws_layout(d, pt->batch, pt->max_pages_per_seq);
+    const bool head_max = mode == kModeDelta && sp->reduce == DELTA_HEAD_MAX;
+    const WsLayout L = ws_layout(d, pt->batch, pt->max_pages_per_seq, head_max);
     if (ws_bytes < L.total) return DELTA_ERR_WORKSPACE;
 
     const int D = d->head_dim, Hq = d->num_q_heads, Hkv = d->num_kv_heads;
@@ -524,6 +527,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.err = reinterpret_cast<int*>(base + L.err);
     prm.o = o;
     prm.num_clusters = plan.clusters;
+    prm.logits = head_max ? reinterpret_cast<float*>(base + L.logits) : nullptr;
     prm.tickets = reinterpret_cast<int*>(base + L.tickets);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -543,6 +547,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     sp2.sel_pages = sel_pages_out;
     sp2.sel_stride = sel_stride_out;
     sp2.page_scores = page_scores;
+    sp2.logits = prm.logits;
     sp2.err = prm.err;
     // one cluster of C CTAs per sequence, about 16K page partials per CTA
     const int maxp = pt->max_pages_per_seq;
@@ -601,6 +606,12 @@ extern "C" {
 size_t delta_workspace_size(const delta_desc* desc, int32_t batch, int32_t max_pages_per_seq) {
     if (check_desc(desc) != DELTA_OK || batch < 0 || max_pages_per_seq < 0) return 0;
     return ws_layout(desc, batch, max_pages_per_seq).total;
+}
+
+size_t delta_workspace_size_reduce(const delta_desc* desc, int32_t batch, int32_t max_pages_per_seq, int32_t reduce) {
+    if (check_desc(desc) != DELTA_OK || batch < 0 || max_pages_per_seq < 0) return 0;
+    if (reduce != DELTA_HEAD_SUM && reduce != DELTA_HEAD_MAX) return 0;
+    return ws_layout(desc, batch, max_pages_per_seq, reduce == DELTA_HEAD_MAX).total;
 }
 
 delta_status delta_workspace_init(void* workspace, size_t ws_bytes, void* stream) {

@@ -17,6 +17,7 @@ struct SelectParams {
     int32_t* sel_pages;
     int32_t sel_stride;
     float* page_scores;
+    const float* logits;   // [B][Hq][max_pages*16] base-2 logits: HEAD_MAX scoring when non-null
     int* err;
 };
 
@@ -156,6 +157,40 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     __syncthreads();
 
     // 2. page scores of this CTA's pages
+    if (p.logits != nullptr) {
+        // HEAD_MAX: S_j = sum over the page's tokens t < n of max_h 2^(s_ht - M_h) / Z_h.  A warp per
+        // page, lanes over heads, each lane holding the page's 16 token maxima of its heads.
+        const size_t hs = size_t(p.max_pages) * kPage;
+        for (int j = j0 + warp; j < j1; j += kSelectThreads / 32) {
+            float mx[kPage];
+#pragma unroll
+            for (int t = 0; t < kPage; ++t) mx[t] = 0.f;
+            for (int h = lane; h < Hq; h += 32) {
+                const float4* lg = reinterpret_cast<const float4*>(p.logits + (size_t(b) * Hq + h) * hs + size_t(j) * kPage);
+                const float inv = 1.f / headZ[h];
+#pragma unroll
+                for (int q4 = 0; q4 < kPage / 4; ++q4) {
+                    const float4 v = lg[q4];
+                    mx[4 * q4 + 0] = fmaxf(mx[4 * q4 + 0], exp2_approx(v.x - headM[h]) * inv);
+                    mx[4 * q4 + 1] = fmaxf(mx[4 * q4 + 1], exp2_approx(v.y - headM[h]) * inv);
+                    mx[4 * q4 + 2] = fmaxf(mx[4 * q4 + 2], exp2_approx(v.z - headM[h]) * inv);
+                    mx[4 * q4 + 3] = fmaxf(mx[4 * q4 + 3], exp2_approx(v.w - headM[h]) * inv);
+                }
+            }
+            float sc = 0.f;
+#pragma unroll
+            for (int t = 0; t < kPage; ++t) {
+                float v = mx[t];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                if (j * kPage + t < n) sc += v;
+            }
+            if (lane == 0) {
+                keys[j - j0] = order_key(sc);
+                if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
+            }
+        }
+    } else
     for (int j = j0 + tid; j < j1; j += kSelectThreads) {
         float sc = 0.f;
         const float2* pm = p.page_ml + size_t(b) * Hq * p.max_pages + j;

@@ -36,7 +36,7 @@ class DeltaStack:
     def __init__(self, kinds, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: torch.dtype,
                  indptr: torch.Tensor, indices: torch.Tensor, kv_len: torch.Tensor, max_pages_per_seq: int,
                  num_phys_pages: int, budget_pages: int = 0, sink_tokens: int = 0, recency_tokens: int = 0,
-                 sm_scale: float = 0.0, keep_scores: bool = False):
+                 sm_scale: float = 0.0, keep_scores: bool = False, reduce: int = N.DELTA_HEAD_SUM):
         self.kinds = list(kinds)
         self.device = indptr.device
         self.batch = int(kv_len.numel())
@@ -48,9 +48,9 @@ class DeltaStack:
         self.indptr, self.indices, self.kv_len = indptr, indices, kv_len
         self.pt = N.DeltaPageTable(indptr.data_ptr(), indices.data_ptr(), kv_len.data_ptr(), self.batch,
                                    max_pages_per_seq)
-        self.sp = N.DeltaSelectParams(budget_pages, sink_tokens, recency_tokens, N.DELTA_HEAD_SUM)
+        self.sp = N.DeltaSelectParams(budget_pages, sink_tokens, recency_tokens, reduce)
         self.max_pages = max_pages_per_seq
-        self.ws_bytes = N.workspace_size(self.desc, self.batch, max_pages_per_seq)
+        self.ws_bytes = N.workspace_size_reduce(self.desc, self.batch, max_pages_per_seq, reduce)
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         N.workspace_init(self.workspace, self.ws_bytes, torch.cuda.current_stream(self.device).cuda_stream)
         self.sel_stride = max(N.sel_capacity(self.sp), 1)

@@ -94,7 +94,13 @@ def test_select_arguments_rejected(L):
     args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
     assert L.select_attn(d, _pt(L), sp, *args[:4], FAKE, FAKE, cap - 1, None, FAKE, ws, 0, check=False) == 1
     sp_max = L.DeltaSelectParams(64, 16, 256, L.DELTA_HEAD_MAX)
-    assert L.select_attn(d, _pt(L), sp_max, *args[:4], FAKE, FAKE, cap, None, FAKE, ws, 0, check=False) == 2
+    ws_max = L.workspace_size_reduce(d, 1, 512, L.DELTA_HEAD_MAX)
+    assert ws_max == ws + 28 * 512 * 16 * 4          # per-token logits of every query head
+    assert L.workspace_size_reduce(d, 1, 512, L.DELTA_HEAD_SUM) == ws
+    assert L.workspace_size_reduce(d, 1, 512, 7) == 0
+    assert L.select_attn(d, _pt(L), sp_max, *args[:4], FAKE, FAKE, cap, None, FAKE, ws, 0, check=False) == 3
+    sp_bad_mode = L.DeltaSelectParams(64, 16, 256, 5)
+    assert L.select_attn(d, _pt(L), sp_bad_mode, *args[:4], FAKE, FAKE, cap, None, FAKE, ws, 0, check=False) == 1
     sp_bad = L.DeltaSelectParams(-1, 16, 256, L.DELTA_HEAD_SUM)
     assert L.select_attn(d, _pt(L), sp_bad, *args[:4], FAKE, FAKE, cap, None, FAKE, ws, 0, check=False) == 1
     assert L.select_attn(d, _pt(L, maxp=40000), sp, *args[:4], FAKE, FAKE, cap, None, FAKE,

@@ -157,13 +157,25 @@ SELECT_CASES = [
 ]
 
 
-@pytest.mark.parametrize("G,Hkv,D,dtype,ctx,k,sink,rec,planted", SELECT_CASES)
-def test_select_attn_matches_oracle(L, G, Hkv, D, dtype, ctx, k, sink, rec, planted):
+MAX_CASES = [
+    (8, 1, 64, "f32", [1024], 8, 16, 64, 0),
+    (7, 4, 128, "bf16", [8192], 64, 16, 256, 32),
+    (4, 2, 128, "bf16", [3000, 1500, 17], 16, 16, 100, 32),
+    (1, 1, 128, "bf16", [777], 5, 16, 32, 8),          # one query head: MAX equals SUM
+]
+
+
+@pytest.mark.parametrize("mode,G,Hkv,D,dtype,ctx,k,sink,rec,planted",
+                         [("sum",) + c for c in SELECT_CASES] + [("max",) + c for c in MAX_CASES])
+def test_select_attn_matches_oracle(L, mode, G, Hkv, D, dtype, ctx, k, sink, rec, planted):
     cfg = make_cfg(G, Hkv, D, dtype, ctx, budget_pages=k, sink=sink, rec=rec, planted=planted)
     dc = device_case(cfg)
     desc, pt = make_desc(L, cfg, dc), make_pt(L, dc)
-    ws, nb = workspace(L, desc, dc)
-    sp = L.DeltaSelectParams(k, sink, rec, L.DELTA_HEAD_SUM)
+    reduce = L.DELTA_HEAD_MAX if mode == "max" else L.DELTA_HEAD_SUM
+    nb = L.workspace_size_reduce(desc, cfg.batch, dc.case.max_pages_per_seq, reduce)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    L.workspace_init(ws, nb, stream())
+    sp = L.DeltaSelectParams(k, sink, rec, reduce)
     stride = L.sel_capacity(sp) + 3
     B, maxp = cfg.batch, dc.case.max_pages_per_seq
     sel_cnt = torch.full((B,), -1, dtype=torch.int32, device="cuda")
@@ -178,8 +190,9 @@ def test_select_attn_matches_oracle(L, G, Hkv, D, dtype, ctx, k, sink, rec, plan
         K, V = oracle_kv(dc.case, 0, b)
         ref, p = O.full_attention(dc.case.q(0)[b].astype(np.float64), K, V)
         assert_close(out[b], ref, dtype, f"o b={b}")
-        S = O.page_scores(p, 16)
-        np.testing.assert_allclose(sc[b, :len(S)], S, rtol=2e-5, atol=1e-6 * cfg.num_q_heads)
+        S = O.page_scores(p, 16, O.HEAD_MAX if mode == "max" else O.HEAD_SUM)
+        np.testing.assert_allclose(sc[b, :len(S)], S, rtol=2e-5 if mode == "sum" else 1e-4,
+                                   atol=1e-6 * cfg.num_q_heads)
         gsel = pages[b, :cnt[b]].tolist()
         ok, exact, ref_sel = selection_ok(gsel, S, n, k, sink, rec)
         assert ok, f"b={b}: gpu {gsel} vs oracle {ref_sel}"
