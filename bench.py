@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
     ap.add_argument("--print-source-hash", action="store_true", help="print the kernel-source hash and exit")
     ap.add_argument("--drift-checks", type=int, default=10, help="oracle selection checks along a trajectory")
+    ap.add_argument("--delta-sweep", type=str, default="",
+                    help="comma list of delta-layer counts: time the step for each (spread placement)")
     return ap.parse_args()
 
 
@@ -544,6 +546,69 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------- delta-layer sweep
+def delta_placement(num_layers: int, m: int) -> list:
+    """m delta-layers, the first at layer 2 (the page's rule) and the rest spread evenly to the end."""
+    span = num_layers - 2
+    return sorted({2 + (i * span) // m for i in range(m)})
+
+
+def run_delta_sweep(args, cfg, counts):
+    """Decode-step time against the number of delta-layers on one workload (one JSON line)."""
+    import torch
+    from long_context_layer_b200.stack import DeltaStack
+    from synth.case import Case
+    from synth.gpu import DeviceCase
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    case = Case(cfg)
+    dc = DeviceCase(case, device=device, prefill="append")
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+    flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    args_step = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+
+    def time_kinds(kinds):
+        st = DeltaStack(kinds, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr, dc.indices,
+                        dc.kv_len, case.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages, cfg.sink_tokens,
+                        cfg.recency_tokens)
+        g = st.capture(*args_step)
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1)
+            flush_rd.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                ts.append(e0.elapsed_time(e1) * 1000.0)
+        del g
+        st.graph = None
+        return statistics.median(ts)
+
+    points = []
+    L = cfg.num_layers
+    full_us = time_kinds(["full"] * L)
+    for m in counts:
+        m = max(1, min(m, L - 2))
+        dl = delta_placement(L, m)
+        c2 = cfg.with_(delta_layers=tuple(dl))
+        tok_delta, tok_full, _, _ = attended_tokens(c2, case)
+        us = time_kinds(c2.layer_kinds())
+        points.append({"delta_layers": dl, "count": len(dl), "us_per_step": round(us, 3),
+                       "speedup_vs_full_stack": round(full_us / us, 3),
+                       "attended_token_reduction": round(tok_full / tok_delta, 3)})
+    print(json.dumps({"metric": "us_per_decode_step_vs_delta_layer_count", "unit": "us/step",
+                      "config": {"workload": cfg.name, "layers": L, "batch": cfg.batch,
+                                 "context": int(case.n.max())},
+                      "full_stack_us": round(full_us, 3), "steps": args.steps, "warmup": args.warmup,
+                      "points": points}), flush=True)
+
+
 def main():
     args = parse()
     if args.print_source_hash:
@@ -554,7 +619,9 @@ def main():
         return
     from synth import configs as C
     cfg = C.CONFIGS[args.config]
-    if cfg.steps > 1:
+    if args.delta_sweep:
+        run_delta_sweep(args, cfg, [int(x) for x in args.delta_sweep.split(",")])
+    elif cfg.steps > 1:
         run_trajectory(args, cfg)
     else:
         run_ours(args)
