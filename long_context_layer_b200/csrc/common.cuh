@@ -194,7 +194,8 @@ struct SeqExtent {
     const int32_t* table;   // the sequence's page-table row staged in shared memory, or null
 };
 
-template <typename P>
+// QUIET: a speculative lookup (before the wait, for an L2 prefetch only) that raises no flags.
+template <bool QUIET = false, typename P>
 __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int b, int i0, int warp, int nk, int kbase,
                                             int lane, int& lp, int& ph) {
     const int k = kbase + lane;
@@ -204,12 +205,13 @@ __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int
     const int i = i0 + warp + k * kWarps;
     lp = (p.mode == kModeSparse) ? p.sel_pages[size_t(b) * p.sel_stride + i] : i;
     if (lp < 0 || lp >= ex.N) {
-        atomicOr(p.err, kErrSel);
+        if (!QUIET) atomicOr(p.err, kErrSel);
+        lp = -1;
         return;
     }
     const int64_t x = ex.table != nullptr ? ex.table[lp] : p.indices[ex.pbeg + lp];
     if (x < 0 || x >= p.num_phys_pages) {
-        atomicOr(p.err, kErrPage);
+        if (!QUIET) atomicOr(p.err, kErrPage);
         return;
     }
     ph = int(x);

@@ -116,24 +116,39 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
         pages_init(pages, p, ex, b, i0, warp, nk, lane);
     };
+    // Before the wait the previous kernel may still be running: warm L2 with the pages this warp
+    // loads first (one pipeline's worth; more would crowd L2 on long contexts) and the group's
+    // queries.  A bulk L2 prefetch is only a cache hint, coherent with
+    // any later write, so prefetching data that is about to change (the current token's slot,
+    // a selection being rewritten) costs bandwidth, never correctness.
+    auto prefetch_page = [&](int ph) {
+        if (ph < 0 || lane >= STAGES) return;
+        const size_t off = (size_t(ph) * p.num_kv_heads + g) * kPage * D;
+        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.k_pool) + off, kPage * D * 2);
+        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.v_pool) + off, kPage * D * 2);
+    };
+    if (threadIdx.x == 0)
+        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t(b) * Hq + h0) * D, G * D * 2);
     if (p.mode != kModeSparse) {
         setup();
-        // Warm L2 with this warp's first pages while the previous kernel drains.  Only the
-        // current token's slot of a pool changes between layers' kernels, and an L2 prefetch is
-        // coherent with later writes, so this is safe before the wait.
-        if (lane < min(STAGES, nk)) {
-            const int ph = pages.ph_a;   // lane j holds page j of the warp
-            if (ph >= 0) {
-                const size_t off = (size_t(ph) * p.num_kv_heads + g) * kPage * D;
-                prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.k_pool) + off, kPage * D * 2);
-                prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.v_pool) + off, kPage * D * 2);
-            }
+        prefetch_page(pages.ph_a);   // lane j holds page j of the warp
+    } else {
+        if (S::kTable > 0 && ex.N <= S::kTable) {
+            // stage the page-table row so that, after the wait, a selected page costs one load
+            for (int j = threadIdx.x; j < ex.N; j += kThreads) table[j] = p.indices[ex.pbeg + j];
+            __syncthreads();
+            ex.table = table;
         }
-    } else if (S::kTable > 0 && ex.N <= S::kTable) {
-        // stage the page-table row so that, after the wait, a selected page costs one load
-        for (int j = threadIdx.x; j < ex.N; j += kThreads) table[j] = p.indices[ex.pbeg + j];
-        __syncthreads();
-        ex.table = table;
+        // Speculate that the selection is already final (it is for every sparse layer but the
+        // first after a delta-layer); the real list is read again after the wait.
+        const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
+        const int scnt = min(max(p.sel_cnt[b], 0), cap);
+        const int si0 = split * p.items_per_split;
+        const int si1 = min(si0 + p.items_per_split, scnt);
+        const int snk = (si1 - si0 > warp) ? (si1 - si0 - warp + kWarps - 1) / kWarps : 0;
+        int slp, sph;
+        fetch_pages<true>(p, ex, b, si0, warp, snk, 0, lane, slp, sph);
+        prefetch_page(sph);
     }
     pdl_wait();      // q, the pools and the selection are written by earlier kernels
     pdl_trigger();
