@@ -118,13 +118,16 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     for (int h = warp; h < Hq; h += kSelectThreads / 32) {
         const float2* pm = p.page_ml + (size_t(b) * Hq + h) * p.max_pages;
         float M = -INFINITY, Z = 0.f;
-        // four independent loads in flight per lane, then an online (max, sum) update
-        for (int j = j0 + lane; j < j1; j += 128) {
-            float2 v[4];
+        // sixteen independent loads in flight per lane, then an online (max, sum) update
+        for (int base = j0; base < j1; base += 32 * 16) {
+            float2 v[16];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = (j + 32 * u < j1) ? pm[j + 32 * u] : make_float2(-INFINITY, 0.f);
+            for (int u = 0; u < 16; ++u) {
+                const int j = base + lane + 32 * u;
+                v[u] = (j < j1) ? pm[j] : make_float2(-INFINITY, 0.f);
+            }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 16; ++u) {
                 const float Mn = fmaxf(M, v[u].x);
                 const float mu = (Mn == -INFINITY) ? 0.f : Mn;
                 Z = Z * exp2_approx(M - mu) + v[u].y * exp2_approx(v[u].x - mu);
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
             M = Mn;
         }
         headM[h] = M;
-        headZ[h] = Z;
+        headZ[h] = 1.f / Z;   // stored as the reciprocal: the score pass multiplies
     }
     __syncthreads();
 
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
             for (int t = 0; t < kPage; ++t) mx[t] = 0.f;
             for (int h = lane; h < Hq; h += 32) {
                 const float4* lg = reinterpret_cast<const float4*>(p.logits + (size_t(b) * Hq + h) * hs + size_t(j) * kPage);
-                const float inv = 1.f / headZ[h];
+                const float inv = headZ[h];
 #pragma unroll
                 for (int q4 = 0; q4 < kPage / 4; ++q4) {
                     const float4 v = lg[q4];
@@ -190,24 +193,34 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
                 if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
             }
         }
-    } else
-    for (int j = j0 + tid; j < j1; j += kSelectThreads) {
-        float sc = 0.f;
-        const float2* pm = p.page_ml + size_t(b) * Hq * p.max_pages + j;
-        int h = 0;
-        for (; h + 8 <= Hq; h += 8) {   // eight independent loads in flight
-            float2 v[8];
+    } else {
+        // HEAD_SUM: two threads per page, each summing every other head with up to sixteen
+        // independent loads in flight, so a page's partials arrive in one round
+        const int sub = tid & 1;
+        for (int base = j0; base < j1; base += kSelectThreads / 2) {   // uniform trip count
+            const int j = base + (tid >> 1);
+            const bool active = j < j1;
+            const float2* pm = p.page_ml + size_t(b) * Hq * p.max_pages + (active ? j : j0);
+            float sc = 0.f;
+            for (int hb = 0; hb < Hq; hb += 32) {
+                float2 v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = pm[size_t(h + u) * p.max_pages];
+                for (int u = 0; u < 16; ++u) {
+                    const int h = hb + sub + 2 * u;
+                    v[u] = (active && h < Hq) ? pm[size_t(h) * p.max_pages] : make_float2(-INFINITY, 0.f);
+                }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) sc += exp2_approx(v[u].x - headM[h + u]) * v[u].y / headZ[h + u];
+                for (int u = 0; u < 16; ++u) {
+                    const int h = hb + sub + 2 * u;
+                    if (h < Hq) sc += exp2_approx(v[u].x - headM[h]) * v[u].y * headZ[h];
+                }
+            }
+            sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+            if (active && sub == 0) {
+                keys[j - j0] = order_key(sc);
+                if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
+            }
         }
-        for (; h < Hq; ++h) {
-            const float2 ml = pm[size_t(h) * p.max_pages];
-            sc += exp2_approx(ml.x - headM[h]) * ml.y / headZ[h];
-        }
-        keys[j - j0] = order_key(sc);
-        if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
     }
     __syncthreads();
 
@@ -223,18 +236,20 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
                 if (!forced(j) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
             }
             __syncthreads();
-            uint32_t* rh = recv_hist + (pass & 1) * C * 256;
-            for (int i = tid; i < C * 256; i += kSelectThreads) {
-                const int j = i >> 8, bin = i & 255;
-                cluster.map_shared_rank(rh, j)[rank * 256 + bin] = hist[bin];
+            if (C > 1) {   // sum the histograms of the cluster (one CTA: already the total)
+                uint32_t* rh = recv_hist + (pass & 1) * C * 256;
+                for (int i = tid; i < C * 256; i += kSelectThreads) {
+                    const int j = i >> 8, bin = i & 255;
+                    cluster.map_shared_rank(rh, j)[rank * 256 + bin] = hist[bin];
+                }
+                cluster_barrier();
+                if (tid < 256) {
+                    uint32_t t = 0;
+                    for (int j = 0; j < C; ++j) t += rh[j * 256 + tid];
+                    hist[tid] = t;
+                }
+                __syncthreads();
             }
-            cluster_barrier();
-            if (tid < 256) {
-                uint32_t t = 0;
-                for (int j = 0; j < C; ++j) t += rh[j * 256 + tid];
-                hist[tid] = t;
-            }
-            __syncthreads();
             if (tid < 32) {
                 // lane covers digits 255-8*lane .. 248-8*lane (descending)
                 uint32_t c[8], sum = 0;
