@@ -116,22 +116,33 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
         pages_init(pages, p, ex, b, i0, warp, nk, lane);
     };
-    // Before the wait the previous kernel may still be running: warm L2 with the pages this warp
-    // loads first (one pipeline's worth; more would crowd L2 on long contexts) and the group's
-    // queries.  A bulk L2 prefetch is only a cache hint, coherent with
-    // any later write, so prefetching data that is about to change (the current token's slot,
-    // a selection being rewritten) costs bandwidth, never correctness.
-    auto prefetch_page = [&](int ph) {
-        if (ph < 0 || lane >= STAGES) return;
-        const size_t off = (size_t(ph) * p.num_kv_heads + g) * kPage * D;
-        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.k_pool) + off, kPage * D * 2);
-        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.v_pool) + off, kPage * D * 2);
+    const uint64_t policy = evict_first_policy();
+    // TMA of one page (K and V of KV head g) into stage k % STAGES; lane 0 only.
+    auto load_page = [&](int k, int ph) {
+        const int s = k % STAGES;
+        unsigned char* dst = wst + size_t(s) * S::kPage;
+        const int y = (ph * p.num_kv_heads + g) * kPage;   // row of (page, KV head g)
+        mbar_expect_tx(&wbar[s], S::kPage);
+#pragma unroll
+        for (int nb = 0; nb < S::kBoxes; ++nb) {
+            tma_load_2d(dst + nb * S::kBox, &tmap_k, nb * 64, y, &wbar[s], policy);
+            tma_load_2d(dst + (S::kBoxes + nb) * S::kBox, &tmap_v, nb * 64, y, &wbar[s], policy);
+        }
     };
+
+    // ---- First pipeline stage, before the wait.  The previous kernel may still be running, so
+    // only data no earlier kernel of the step changes is loaded now: pool pages other than the
+    // sequence's last one (the appended token's page is loaded after the wait).  Full and delta
+    // layers know their pages; sparse layers speculate that the selection is already final (it
+    // is for every sparse layer but the first after a delta-layer) and check it after the wait.
     if (threadIdx.x == 0)
         prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t(b) * Hq + h0) * D, G * D * 2);
+    uint32_t early = 0;       // bit k: page k's load was issued before the wait
+    uint32_t spec_used = 0;   // bit s: stage s spent its first phase on a discarded speculative load
+    WarpPages spec;
+    int nk_spec = 0;
     if (p.mode != kModeSparse) {
         setup();
-        prefetch_page(pages.ph_a);   // lane j holds page j of the warp
     } else {
         if (S::kTable > 0 && ex.N <= S::kTable) {
             // stage the page-table row so that, after the wait, a selected page costs one load
@@ -139,22 +150,32 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
             __syncthreads();
             ex.table = table;
         }
-        // Speculate that the selection is already final (it is for every sparse layer but the
-        // first after a delta-layer); the real list is read again after the wait.
         const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
         const int scnt = min(max(p.sel_cnt[b], 0), cap);
         const int si0 = split * p.items_per_split;
         const int si1 = min(si0 + p.items_per_split, scnt);
-        const int snk = (si1 - si0 > warp) ? (si1 - si0 - warp + kWarps - 1) / kWarps : 0;
-        int slp, sph;
-        fetch_pages<true>(p, ex, b, si0, warp, snk, 0, lane, slp, sph);
-        prefetch_page(sph);
+        nk_spec = (si1 - si0 > warp) ? (si1 - si0 - warp + kWarps - 1) / kWarps : 0;
+        spec.cur = 0;
+        fetch_pages<true>(p, ex, b, si0, warp, nk_spec, 0, lane, spec.lp_a, spec.ph_a);
+        spec.lp_b = spec.ph_b = -1;
     }
-    pdl_wait();      // q, the pools and the selection are written by earlier kernels
+    {
+        const WarpPages& pre = (p.mode == kModeSparse) ? spec : pages;
+        const int npre = min(STAGES, (p.mode == kModeSparse) ? nk_spec : nk);
+        for (int k = 0; k < npre; ++k) {
+            int lp, ph;
+            pages_get(pre, k, lp, ph);
+            if (ph >= 0 && lp != ex.N - 1) {
+                if (lane == 0) load_page(k, ph);
+                early |= 1u << k;
+            }
+        }
+    }
+    pdl_wait();      // q, the appended token, and a selection written by the previous kernel
     pdl_trigger();
-    if (p.mode == kModeSparse) setup();
 
-    // ---- Q^T fragments (B operand of the QK product): head g4 of the group, dims k*16 + 2*t4 (+8)
+    // ---- Q^T fragments (B operand of the QK product): head g4 of the group, dims k*16 + 2*t4 (+8);
+    // issued first so their latency overlaps the selection check below
     uint32_t qb[KS][2];
     {
         const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t(b) * Hq + h0 + g4) * D;
@@ -169,27 +190,55 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         }
     }
 
-    const uint64_t policy = evict_first_policy();
+    if (p.mode == kModeSparse) {
+        seq_count(p, b, ex);
+        i0 = split * p.items_per_split;
+        const int i1 = min(i0 + p.items_per_split, ex.count);
+        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;
+        // The speculation holds if the selection's logical pages of this warp's first chunk are the
+        // ones guessed (the page table does not change within the step) and were all valid.
+        const int lp_real = (lane < nk) ? p.sel_pages[size_t(b) * p.sel_stride + i0 + warp + lane * kWarps] : -1;
+        const bool all_same = __all_sync(0xffffffffu, lane >= nk || (lp_real == spec.lp_a && spec.ph_a >= 0)) &&
+                              nk == nk_spec;
+        if (all_same) {
+            pages = spec;
+            fetch_pages(p, ex, b, i0, warp, nk, 32, lane, pages.lp_b, pages.ph_b);
+        } else {
+            pages_init(pages, p, ex, b, i0, warp, nk, lane);
+            // keep an early load only if it is exactly the selection's page; otherwise drain all
+            bool same = nk == nk_spec;
+            for (int k = 0; k < min(STAGES, nk_spec); ++k) {
+                if (!((early >> k) & 1u)) continue;
+                int lp0, ph0, lp1, ph1;
+                pages_get(spec, k, lp0, ph0);
+                pages_get(pages, k, lp1, ph1);
+                same = same && lp0 == lp1 && ph0 == ph1;
+            }
+            if (!same) {
+                // drain the speculative loads (bounded wait); those stages start their real use one
+                // phase later
+                for (int k = 0; k < min(STAGES, nk_spec); ++k)
+                    if ((early >> k) & 1u) {
+                        if (!mbar_wait(&wbar[k % STAGES], 0) && lane == 0) atomicOr(p.err, kErrTimeout);
+                        spec_used |= 1u << (k % STAGES);
+                    }
+                early = 0;
+            }
+        }
+    }
+
     // all lanes call (the page id is shuffled out of the prefetched list); lane 0 issues
     auto issue = [&](int k) {
         int lp, ph;
         pages_get(pages, k, lp, ph);
         if (lane != 0) return;
-        const int s = k % STAGES;
-        if (ph >= 0) {
-            unsigned char* dst = wst + size_t(s) * S::kPage;
-            const int y = (ph * p.num_kv_heads + g) * kPage;   // row of (page, KV head g)
-            mbar_expect_tx(&wbar[s], S::kPage);
-#pragma unroll
-            for (int nb = 0; nb < S::kBoxes; ++nb) {
-                tma_load_2d(dst + nb * S::kBox, &tmap_k, nb * 64, y, &wbar[s], policy);
-                tma_load_2d(dst + (S::kBoxes + nb) * S::kBox, &tmap_v, nb * 64, y, &wbar[s], policy);
-            }
-        } else {
-            mbar_arrive(&wbar[s]);   // completes the phase with no data; the page is skipped
-        }
+        if (ph >= 0) load_page(k, ph);
+        else mbar_arrive(&wbar[k % STAGES]);   // completes the phase with no data; the page is skipped
     };
-    for (int k = 0; k < min(STAGES, nk); ++k) issue(k);
+    for (int k = 0; k < min(STAGES, nk); ++k)
+        if (!((early >> k) & 1u)) issue(k);
+    // phase parity of the stage holding page k
+    auto parity = [&](int k) -> uint32_t { return ((k / STAGES) + ((spec_used >> (k % STAGES)) & 1u)) & 1u; };
 
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2*t4, 2*t4+1
     float acc[KS][4];
@@ -281,7 +330,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         pages_advance(pages, p, ex, b, i0, warp, nk, lane, k);
         const bool two = k + 1 < nk;
         const int sA = k % STAGES, sB = (k + 1) % STAGES;
-        if (!mbar_wait(&wbar[sA], (k / STAGES) & 1) || (two && !mbar_wait(&wbar[sB], ((k + 1) / STAGES) & 1))) {
+        if (!mbar_wait(&wbar[sA], parity(k)) || (two && !mbar_wait(&wbar[sB], parity(k + 1)))) {
             if (lane == 0) atomicOr(p.err, kErrTimeout);
             failed = true;
             break;
@@ -350,7 +399,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     }
     if (failed) {
         // drain this warp's copies still in flight (bounded) before shared memory is released
-        for (int k = consumed + 1; k < min(consumed + STAGES, nk); ++k) mbar_wait(&wbar[k % STAGES], (k / STAGES) & 1);
+        for (int k = consumed + 1; k < min(consumed + STAGES, nk); ++k) mbar_wait(&wbar[k % STAGES], parity(k));
     }
 
     // ---- merge the 4 warps' states of this CTA, then the splits

@@ -134,7 +134,15 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
     SplitPlan pl;
     pl.cluster = s < 16 ? s : 16;
     pl.clusters = s / pl.cluster;
-    pl.deep = dtype == DELTA_BF16 && int64_t(units) * pl.splits() <= sms;
+    // The deep variant (6 stages, one CTA per SM) leaves no room on an SM for the next layer's
+    // CTAs, which then cannot start their first loads while this layer drains; the shallow one
+    // (3 stages, two CTAs per SM) can, and measured faster on every workload, so deep is opt-in.
+    static int deep = -1;
+    if (deep < 0) {
+        const char* e = getenv("DELTA_DEEP");   // tuning override for sweeps
+        deep = (e != nullptr && atoi(e) > 0) ? 1 : 0;
+    }
+    pl.deep = deep && dtype == DELTA_BF16 && int64_t(units) * pl.splits() <= sms;
     return pl;
 }
 
