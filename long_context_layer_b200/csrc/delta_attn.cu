@@ -340,9 +340,15 @@ int max_active_clusters(const void* func, size_t smem, int cluster) {
 // into the GPCs.
 SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) {
     const int s = pl.splits();
-    // Clusters meet through the workspace only when each gets at least 256 pages: below that the
-    // cross-cluster merge costs more than the extra CTAs gain.
-    const int max_clusters = items / 256 > 1 ? items / 256 : 1;
+    // Clusters meet through the workspace only when each gets at least 256 pages (and the unit has
+    // more than 512): below that the cross-cluster merge costs more than the extra CTAs gain.
+    static int per_cluster = -1;
+    if (per_cluster < 0) {
+        const char* e = getenv("DELTA_PAGES_PER_CLUSTER");   // tuning override for sweeps
+        per_cluster = (e != nullptr && atoi(e) > 0) ? atoi(e) : 256;
+    }
+    // Up to 512 pages per (sequence, KV head) one cluster is faster (measured on the 8k stack).
+    const int max_clusters = (items <= 512 || items / per_cluster < 1) ? 1 : items / per_cluster;
     SplitPlan best = pl;
     int best_ctas = -1;
     for (int c = pl.cluster; c >= 1; --c) {
