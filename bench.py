@@ -479,7 +479,13 @@ def run_ours(args):
     qo_bytes = 2 * cfg.batch * cfg.num_q_heads * cfg.head_dim * e
     alg_bytes = kv_bytes + qo_bytes
     peak, peak_kind = load_peaks()
-    achieved = alg_bytes / (us_kernel * 1e-6) / 1e9
+    # The full-attention stack is one graph of L launches of this same decode kernel (plus one
+    # append launch), timed with CUDA events: its per-launch average is the kernel's duration in
+    # steady state (the append is charged to it, which only lowers the figure).  The single call
+    # timed above also carries a launch latency no graph pays; it is reported alongside.
+    us_launch = us_full / cfg.num_layers
+    achieved = alg_bytes / (us_launch * 1e-6) / 1e9
+    achieved_single = alg_bytes / (us_kernel * 1e-6) / 1e9
 
     # -- end to end through the public API: pinned host inputs in, outputs out, every step
     q_h = dc.q.cpu().pin_memory()
@@ -526,10 +532,13 @@ def run_ours(args):
             "full_stack_us": round(us_full, 3),
             "speedup_vs_full_stack": round(us_full / us_delta, 3),
             "attended_token_reduction": round(tok_full / tok_delta, 3),
-            "roofline": {"kernel": "decode_kernel (full layer, fused split merge)", "bound": "hbm",
+            "roofline": {"kernel": "decode_mma_kernel, full layer (split-KV, cluster merge)", "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                         "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_kernel, 3),
+                         "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_launch, 3),
+                         "timing": "full-attention stack graph (L launches + 1 append) / L, CUDA events, L2 flushed",
+                         "single_call_us": round(us_kernel, 3),
+                         "single_call_frac": round(achieved_single / peak, 4),
                          "traffic": profiled_traffic(cfg.name)},
             "breakdown_us_per_call": breakdown,
             "e2e": {"value": round(us_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

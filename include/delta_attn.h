@@ -198,6 +198,15 @@ delta_status delta_sparse_attn(const delta_desc* desc, const delta_page_table* p
                                const void* q, const void* k_pool, const void* v_pool, void* o,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* Delta-layer calibration metric: shift_out[b] = 1 - cos(scores_a[b], scores_b[b]) over the
+ * pages j < ceil(kv_len[b]/page_size) of two layers' page scores (the page_scores outputs of
+ * delta_select_attn, [batch][max_pages_per_seq] fp32).  The calibration picks delta-layers
+ * from the average shift between consecutive layers, "1 - cosine similarity averaged over
+ * decoding steps and samples" (ai.info summary, "Methodology in Plain English"); a layer's
+ * attention map is read as its page-score vector.  A zero vector gives a shift of 1. */
+delta_status delta_layer_shift(const delta_page_table* pt, const float* scores_a, const float* scores_b,
+                               float* shift_out, void* stream);
+
 /* Synchronise `stream`, read and clear the workspace's device error flags.
  * Returns DELTA_OK, DELTA_ERR_BOUNDS (a device-side check failed since the last
  * read) or DELTA_ERR_CUDA.  *flags_out (nullable) receives the raw flag bits:

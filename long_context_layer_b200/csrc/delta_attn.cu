@@ -726,6 +726,16 @@ delta_status delta_sparse_attn(const delta_desc* desc, const delta_page_table* p
                          nullptr, 0, nullptr, workspace, ws_bytes, stream);
 }
 
+delta_status delta_layer_shift(const delta_page_table* pt, const float* scores_a, const float* scores_b,
+                               float* shift_out, void* stream) {
+    delta_status s = check_pt(pt);
+    if (s != DELTA_OK) return s;
+    if (pt->batch == 0) return DELTA_OK;
+    if (scores_a == nullptr || scores_b == nullptr || shift_out == nullptr) return DELTA_ERR_INVALID_ARG;
+    return launch_pdl(layer_shift_kernel, dim3(pt->batch), dim3(kShiftThreads), 0, static_cast<cudaStream_t>(stream),
+                      scores_a, scores_b, pt->page_indptr, pt->kv_len, pt->max_pages_per_seq, shift_out);
+}
+
 delta_status delta_read_device_error(void* workspace, int32_t* flags_out, void* stream) {
     if (workspace == nullptr) return DELTA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

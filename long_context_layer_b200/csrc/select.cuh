@@ -332,6 +332,45 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     if (rank == 0 && tid == 0) p.sel_cnt[b] = min(total, p.sel_stride);
 }
 
+// ------------------------------------------------------------------ layer-shift metric
+// 1 - cos(S_a[b], S_b[b]) over the pages j < ceil(kv_len[b]/16) of two layers' page scores, one
+// CTA per sequence (fixed-order reduction: deterministic).  A zero vector gives 1.
+constexpr int kShiftThreads = 256;
+__global__ void __launch_bounds__(kShiftThreads) layer_shift_kernel(const float* __restrict__ sa,
+                                                                  const float* __restrict__ sb,
+                                                                  const int32_t* __restrict__ indptr,
+                                                                  const int32_t* __restrict__ kv_len, int max_pages,
+                                                                  float* __restrict__ out) {
+    __shared__ float red[3][kShiftThreads / 32];
+    pdl_wait();
+    pdl_trigger();
+    const int b = blockIdx.x, tid = threadIdx.x;
+    int n = kv_len[b];
+    const int npg = indptr[b + 1] - indptr[b];
+    n = min(max(n, 0), max(npg, 0) * kPage);
+    const int N = min((n + kPage - 1) / kPage, max_pages);
+    float ab = 0.f, aa = 0.f, bb = 0.f;
+    for (int j = tid; j < N; j += kShiftThreads) {
+        const float x = sa[size_t(b) * max_pages + j], y = sb[size_t(b) * max_pages + j];
+        ab = fmaf(x, y, ab);
+        aa = fmaf(x, x, aa);
+        bb = fmaf(y, y, bb);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        ab += __shfl_xor_sync(0xffffffffu, ab, o);
+        aa += __shfl_xor_sync(0xffffffffu, aa, o);
+        bb += __shfl_xor_sync(0xffffffffu, bb, o);
+    }
+    if ((tid & 31) == 0) { red[0][tid >> 5] = ab; red[1][tid >> 5] = aa; red[2][tid >> 5] = bb; }
+    __syncthreads();
+    if (tid == 0) {
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+        for (int w = 0; w < kShiftThreads / 32; ++w) { s0 += red[0][w]; s1 += red[1][w]; s2 += red[2][w]; }
+        out[b] = (s1 > 0.f && s2 > 0.f) ? 1.f - s0 / (sqrtf(s1) * sqrtf(s2)) : 1.f;
+    }
+}
+
 // ------------------------------------------------------------------ kv append kernels
 // Copy one token row (row_vecs 16-byte vectors) of KV head g of sequence b into slot
 // (kv_len-1) % 16 of logical page (kv_len-1) / 16.  Out-of-range pages are skipped (the attention

@@ -108,3 +108,44 @@ class DeltaStack:
         cnt = self.sel_cnt[delta_index].cpu().tolist()
         pages = self.sel_pages[delta_index].cpu()
         return [pages[b, :cnt[b]].tolist() for b in range(self.batch)]
+
+    # ------------------------------------------------------------------ calibration
+    def calibration_shifts(self, q, k_pools, v_pools, out, stream: int | None = None) -> torch.Tensor:
+        """Per-layer shift [L, B]: shift[l][b] = 1 - cos(page scores of layer l-1, of layer l).
+
+        Every layer from 1 on runs as a delta-layer (full attention plus page scores) on the
+        current cache; layers 0 and 1 get shift 0.  DELTA's calibration (ai.info summary,
+        "Methodology in Plain English") averages such shifts over decoding steps and samples
+        and places the delta-layers where they are large.
+        """
+        st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
+        L = len(self.kinds)
+        scores = torch.zeros(L, self.batch, self.max_pages, dtype=torch.float32, device=self.device)
+        shift = torch.zeros(L, self.batch, dtype=torch.float32, device=self.device)
+        sel_cnt = torch.zeros(self.batch, dtype=torch.int32, device=self.device)
+        sel_pages = torch.zeros(self.batch, self.sel_stride, dtype=torch.int32, device=self.device)
+        for l in range(1, L):
+            N.select_attn(self.desc, self.pt, self.sp, q[l], k_pools[l], v_pools[l], out[l], sel_cnt, sel_pages,
+                          self.sel_stride, scores[l], self.workspace, self.ws_bytes, st)
+            if l >= 2:
+                N.layer_shift(self.pt, scores[l - 1], scores[l], shift[l], st)
+        return shift
+
+
+def choose_delta_layers(shift, count: int, first: int = 2, min_gap: int = 2) -> list:
+    """Delta-layer placement from per-layer shifts (shift[l]: between layers l-1 and l).
+
+    Layer `first` opens the list (DELTA places its first delta-layer at layer 2; ai.info
+    summary, "Methodology in Plain English"); further layers are added by decreasing shift
+    (equal shifts: lower layer first) when at least `min_gap` layers from every layer already
+    in the list, so large shifts are covered without clustering in depth.
+    """
+    shift = [float(x) for x in shift]
+    chosen = [first]
+    order = sorted(range(first + 1, len(shift)), key=lambda l: (-shift[l], l))
+    for l in order:
+        if len(chosen) >= count:
+            break
+        if min(abs(l - c) for c in chosen) >= min_gap:
+            chosen.append(l)
+    return sorted(chosen)

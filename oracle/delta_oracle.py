@@ -177,3 +177,37 @@ def stack_step(kinds, q_of, kv_of, n: int, page_size: int, budget_pages: int,
         if want:
             outs[l] = o
     return outs, sels
+
+
+def layer_shift(scores_a: np.ndarray, scores_b: np.ndarray) -> float:
+    """Inter-layer shift 1 - cos(S_a, S_b) of two layers' page-score vectors.
+
+    The calibration of the delta-layers (ai.info summary, "Methodology in Plain English") averages
+    1 - cosine similarity between consecutive layers' attention; the page-level attention map of a
+    layer is read here as its vector of page scores.  Zero vectors give a shift of 1.
+    """
+    a = np.asarray(scores_a, dtype=np.float64)
+    b = np.asarray(scores_b, dtype=np.float64)
+    na, nb = np.sqrt((a * a).sum()), np.sqrt((b * b).sum())
+    if na == 0.0 or nb == 0.0:
+        return 1.0
+    return 1.0 - float((a * b).sum() / (na * nb))
+
+
+def choose_delta_layers(shift: np.ndarray, count: int, first: int = 2, min_gap: int = 2) -> list:
+    """Delta-layer placement from per-layer shifts (shift[l] = shift between layers l-1 and l).
+
+    Reading of the calibration step (ai.info summary, "Methodology in Plain English"): the page
+    fixes layer 2 as the first delta-layer and asks for the rest at layers of large shift spread
+    over the depth of the model.  Here layer `first` is taken, then candidates in decreasing
+    shift order (equal shifts: lower layer first), each kept when it lies at least `min_gap`
+    layers from every layer already kept, until `count` layers are kept.
+    """
+    L = len(shift)
+    chosen = [first]
+    for l in sorted(range(first + 1, L), key=lambda l: (-shift[l], l)):
+        if len(chosen) >= count:
+            break
+        if all(abs(l - c) >= min_gap for c in chosen):
+            chosen.append(l)
+    return sorted(chosen)

@@ -272,3 +272,28 @@ def test_delta_selection_recovers_planted_pages():
     _, p = O.full_attention(q, K, rand(Hkv, n, D), 1.0)
     sel = O.select_pages(O.page_scores(p, 16), n, 16, 3, 16, 32)
     assert sel == [0, 3, 8, 13, 23, 24]
+
+
+# ----------------------------------------------------------------- layer-shift calibration
+def test_layer_shift_closed_forms():
+    x = np.array([3.0, 1.0, 0.0, 2.0])
+    assert abs(O.layer_shift(x, x)) < 1e-15
+    assert abs(O.layer_shift(x, 5 * x)) < 1e-15                     # scale invariant
+    assert abs(O.layer_shift([1, 0, 0], [0, 2, 0]) - 1.0) < 1e-15   # orthogonal
+    assert abs(O.layer_shift([1, 0], [1, 1]) - (1 - 1 / math.sqrt(2))) < 1e-15
+    assert O.layer_shift([0, 0], [1, 2]) == 1.0
+
+
+def test_layer_shift_matches_library_cosine():
+    a, b = RNG.random(300), RNG.random(300)
+    ref = 1 - torch.nn.functional.cosine_similarity(torch.from_numpy(a), torch.from_numpy(b), dim=0).item()
+    assert abs(O.layer_shift(a, b) - ref) < 1e-12
+
+
+def test_choose_delta_layers_rules():
+    shift = np.array([0, 0, 0.1, 0.9, 0.85, 0.2, 0.7, 0.1, 0.8])
+    assert O.choose_delta_layers(shift, 1) == [2]
+    # 3 is the largest shift but is adjacent to 2; 8 and 6 follow (4 too close to 3? 3 is not chosen)
+    assert O.choose_delta_layers(shift, 3, min_gap=2) == [2, 4, 8]
+    assert O.choose_delta_layers(shift, 4, min_gap=2) == [2, 4, 6, 8]
+    assert O.choose_delta_layers(shift, 3, min_gap=1) == [2, 3, 4]
