@@ -77,6 +77,28 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 // Bulk prefetch of a global range into L2 (no shared-memory destination, no completion).
+// Distributed shared memory: the cluster address of a shared variable in CTA `rank`, and an
+// asynchronous 8- or 16-byte store into it whose arrival is counted (in bytes) on that CTA's mbarrier.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_async(uint32_t dst, float4 v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(dst),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async(uint32_t dst, float2 v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(dst),
+                 "f"(v.x), "f"(v.y), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
@@ -278,9 +300,23 @@ __device__ __forceinline__ void seq_count(const P& p, int b, SeqExtent& ex) {
 }
 
 // Floats of the dedicated receive area of the cluster merge (never aliased with pipeline stages,
-// so other CTAs of the cluster may push into it while this CTA is still streaming pages).
+// so other CTAs of the cluster may push into it while this CTA is still streaming pages).  Its
+// first 16 bytes hold the mbarrier that counts the bytes pushed into it.
 template <int D>
-constexpr int recv_floats() { return kMaxGroup * D + 16 * 4 + 16 * kMaxGroup * 2 + kMaxGroup * 2; }
+constexpr int recv_floats() { return 4 + kMaxGroup * D + 16 * 4 + 16 * kMaxGroup * 2 + kMaxGroup * 2; }
+
+// Kernel prologue of the cluster merge, all threads, before any page work: thread 0 initialises
+// this CTA's receive barrier, then every thread arrives (relaxed) on the cluster barrier that the
+// epilogue waits on before its first remote store, so no CTA signals a barrier that its owner has
+// not initialised yet.  The wait is long satisfied when the epilogue reaches it.
+__device__ __forceinline__ void merge_prologue(float* recv) {
+    if (threadIdx.x == 0) {
+        mbar_init(reinterpret_cast<uint64_t*>(recv), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    cluster_arrive_relaxed();
+}
 
 template <typename T, int D, int G, int NPART>
 __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
@@ -298,12 +334,17 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
     T* out = reinterpret_cast<T*>(p.o);
 
     // 1. this CTA's NPART states -> one state, pushed straight into the shared memory of the
-    //    cluster CTA that owns each output element (remote stores need no round trip).  Slices
-    //    are multiples of 4 elements so every push is one 16-byte store.
+    //    cluster CTA that owns each output element with asynchronous remote stores; each owner
+    //    waits on its own barrier for the bytes of all C CTAs (no cluster-wide barrier, no round
+    //    trip).  Slices are multiples of 4 elements so every push is one 16-byte store.
     const int total = G * D;
     const int chunk = (((total + C - 1) / C) + 3) & ~3;
+    uint64_t* rbar = reinterpret_cast<uint64_t*>(recv);
+    recv += 4;
     float* recv_ml = recv + C * chunk;                                             // [C][G][2]
     float* cml = recv_ml + C * G * 2;                                              // [G][2] this CTA
+    const int e0 = rank * chunk, e1 = min(e0 + chunk, total);                      // this CTA's slice
+    if (tid == 0) mbar_expect_tx(rbar, uint32_t(C) * (uint32_t(max(e1 - e0, 0)) * 4u + uint32_t(G) * 8u));
     if (tid < G) {
         float M = -INFINITY;
 #pragma unroll
@@ -317,10 +358,11 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
         cml[2 * tid + 1] = L;
     }
     __syncthreads();
+    cluster_wait();   // every CTA of the cluster has initialised its receive barrier
     if (tid < C * G) {   // this CTA's (max, sum) of head h to cluster rank j
         const int j = tid / G, h = tid % G;
-        reinterpret_cast<float2*>(cluster.map_shared_rank(recv_ml, j))[rank * G + h] =
-            make_float2(cml[2 * h], cml[2 * h + 1]);
+        st_async(cluster_addr(recv_ml + (rank * G + h) * 2, j), make_float2(cml[2 * h], cml[2 * h + 1]),
+                 cluster_addr(rbar, j));
     }
     for (int q4 = tid; q4 * 4 < total; q4 += nthr) {
         const int idx = q4 * 4, h = idx / D, d = idx % D;    // D is a multiple of 4: one head per group
@@ -337,12 +379,12 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
             acc.w = fmaf(w, v.w, acc.w);
         }
         const int owner = idx / chunk;
-        *reinterpret_cast<float4*>(cluster.map_shared_rank(recv, owner) + rank * chunk + (idx - owner * chunk)) = acc;
+        st_async(cluster_addr(recv + rank * chunk + (idx - owner * chunk), owner), acc, cluster_addr(rbar, owner));
     }
-    cluster.sync();   // release/acquire: every pushed value is visible to its owner
+    // all C CTAs' bytes have landed (bounded wait; a timeout is flagged and the merge goes on)
+    if (!mbar_wait(rbar, 0) && tid == 0) atomicOr(p.err, kErrTimeout);
 
     // 2. each CTA merges the C states of its slice from its own shared memory
-    const int e0 = rank * chunk, e1 = min(e0 + chunk, total);
     for (int e = e0 + tid; e < e1; e += nthr) {
         const int h = e / D, d = e % D;
         float M = -INFINITY;

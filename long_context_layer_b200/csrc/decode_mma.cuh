@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
     }
     __syncwarp();
+    merge_prologue(recv);
     // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
     // so full and delta layers resolve their pages before waiting for the previous kernel; the
     // sparse layers' page list is the output of the delta-layer and is read after the wait.

@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         fence_mbar_init();
     }
     __syncwarp();
+    merge_prologue(recv);
     // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
     // so full and delta layers resolve their pages before waiting for the previous kernel; the
     // sparse layers' page list is the output of the delta-layer and is read after the wait.
