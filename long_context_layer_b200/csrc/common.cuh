@@ -16,6 +16,7 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxGroup = 8;
 constexpr int kMaxSelectPages = 32768;
+constexpr int kMaxSelectChunk = 16384;   // pages one CTA of the selection cluster owns at most
 constexpr int kSelectThreads = 1024;
 constexpr int kMaxQHeadsSelect = 256;   // query heads a delta-layer selection supports
 constexpr int kMaxSplits = 512;   // the merge stages G*S*12 bytes of split weights in shared memory
@@ -108,6 +109,11 @@ __device__ __forceinline__ float exp2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+__device__ __forceinline__ float log2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // ------------------------------------------------------------------ element access
 template <typename T>
@@ -182,7 +188,8 @@ struct DecodeParams {
     int32_t mode;
     float2* part_ml;  // [B][Hq][S]  (max, sum) of each split, base-2 logits
     float* part_o;    // [B][Hq][S][D] unnormalised outputs of each split
-    float2* page_ml;  // [B][Hq][max_pages] per-page (max, sum) for delta-layers
+    float* page_lse;  // [B][Hq][max_pages] per-page log2-sum-exp of base-2 logits (delta-layers)
+    float2* split_ml; // [B][Hq][S] (max, sum) of each split CTA's own pages (delta-layers)
     void* o;          // [B][Hq][D] output
     int32_t num_clusters;   // clusters along the split dimension (num_splits = cluster size * this)
     float* logits;          // [B][Hq][max_pages*16] base-2 logits (delta-layers in HEAD_MAX mode), else null
@@ -320,7 +327,8 @@ __device__ __forceinline__ void merge_prologue(float* recv) {
 
 template <typename T, int D, int G, int NPART>
 __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
-                                               const float* mml, float* recv, int b, int g) {
+                                               const float* mml, float* recv, int b, int g,
+                                               const float* dml = nullptr) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
@@ -356,6 +364,22 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
             L = fmaf(exp2_approx(mml[(rr * kMaxGroup + tid) * 2] - mu), mml[(rr * kMaxGroup + tid) * 2 + 1], L);
         cml[2 * tid] = M;
         cml[2 * tid + 1] = L;
+        if (p.split_ml != nullptr) {
+            // the selection's per-head totals are combined from these; dml (when given) holds the
+            // parts' states over the exact page terms
+            float Md = M, Ld = L;
+            if (dml != nullptr) {
+                Md = -INFINITY;
+#pragma unroll
+                for (int rr = 0; rr < NPART; ++rr) Md = fmaxf(Md, dml[(rr * kMaxGroup + tid) * 2]);
+                const float md = (Md == -INFINITY) ? 0.f : Md;
+                Ld = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < NPART; ++rr)
+                    Ld = fmaf(exp2_approx(dml[(rr * kMaxGroup + tid) * 2] - md), dml[(rr * kMaxGroup + tid) * 2 + 1], Ld);
+            }
+            p.split_ml[(size_t(b) * Hq + h0 + tid) * p.num_splits + blockIdx.x] = make_float2(Md, Ld);
+        }
     }
     __syncthreads();
     cluster_wait();   // every CTA of the cluster has initialised its receive barrier

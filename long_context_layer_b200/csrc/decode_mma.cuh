@@ -242,6 +242,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     auto parity = [&](int k) -> uint32_t { return ((k / STAGES) + ((spec_used >> (k % STAGES)) & 1u)) & 1u; };
 
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2*t4, 2*t4+1
+    // delta-layers: the same state over the pages' fp32 terms (l_run sums the bf16-rounded
+    // probabilities that also weight V), so the selection's normalisers match its page terms
+    float dm_run[2] = {-INFINITY, -INFINITY}, dl_run[2] = {0.f, 0.f};
     float acc[KS][4];
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
@@ -298,9 +301,14 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
             e0 += __shfl_xor_sync(0xffffffffu, e0, o);
             e1 += __shfl_xor_sync(0xffffffffu, e1, o);
         }
+        const float n0 = fmaxf(dm_run[0], mx0), n1 = fmaxf(dm_run[1], mx1);   // finite: the page is valid
+        dl_run[0] = dl_run[0] * exp2_approx(dm_run[0] - n0) + e0 * exp2_approx(mx0 - n0);
+        dl_run[1] = dl_run[1] * exp2_approx(dm_run[1] - n1) + e1 * exp2_approx(mx1 - n1);
+        dm_run[0] = n0;
+        dm_run[1] = n1;
         const int hA = 2 * t4, hB = 2 * t4 + 1;
-        if (g4 == 0 && hA < G) p.page_ml[(size_t(b) * Hq + h0 + hA) * p.max_pages + lp] = make_float2(mx0, e0);
-        if (g4 == 0 && hB < G) p.page_ml[(size_t(b) * Hq + h0 + hB) * p.max_pages + lp] = make_float2(mx1, e1);
+        if (g4 == 0 && hA < G) p.page_lse[(size_t(b) * Hq + h0 + hA) * p.max_pages + lp] = mx0 + log2_approx(e0);
+        if (g4 == 0 && hB < G) p.page_lse[(size_t(b) * Hq + h0 + hB) * p.max_pages + lp] = mx1 + log2_approx(e1);
     };
     // tokens past the end of the context: zero their V rows (they may hold non-finite bytes)
     auto zero_tail = [&](int s, int tv) {
@@ -415,14 +423,21 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         mo[(warp * kMaxGroup + 2 * t4) * D + d + 8] = acc[mt][2];
         mo[(warp * kMaxGroup + 2 * t4 + 1) * D + d + 8] = acc[mt][3];
     }
+    float* dml = mml + kWarps * kMaxGroup * 2;           // [4][8][2] delta-layers
     if (g4 == 0) {
         mml[(warp * kMaxGroup + 2 * t4) * 2 + 0] = m_run[0];
         mml[(warp * kMaxGroup + 2 * t4) * 2 + 1] = l_run[0];
         mml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 0] = m_run[1];
         mml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 1] = l_run[1];
+        if (p.mode == kModeDelta) {
+            dml[(warp * kMaxGroup + 2 * t4) * 2 + 0] = dm_run[0];
+            dml[(warp * kMaxGroup + 2 * t4) * 2 + 1] = dl_run[0];
+            dml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 0] = dm_run[1];
+            dml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 1] = dl_run[1];
+        }
     }
     __syncthreads();
-    merge_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo, mml, recv, b, g);
+    merge_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo, mml, recv, b, g, dml);
 }
 
 }  // namespace delta

@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 for (int j = 0; j < 8; ++j) e += exp2_approx(sc[j] - mp);
                 e += __shfl_xor_sync(0xffffffffu, e, 16);
                 if (half == 0 && hl < G)
-                    p.page_ml[(size_t(b) * Hq + h0 + hl) * p.max_pages + lp] = make_float2(mp, e);
+                    p.page_lse[(size_t(b) * Hq + h0 + hl) * p.max_pages + lp] = mp + log2_approx(e);
                 if (p.logits != nullptr && hl < G) {   // per-token logits (HEAD_MAX scoring)
                     float* lg = p.logits + ((size_t(b) * Hq + h0 + hl) * p.max_pages + lp) * kPage + half * 8;
 #pragma unroll

@@ -49,7 +49,7 @@ constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB 
 constexpr int kMmaStagesDeep = 6;  // when the whole grid fits one CTA per SM: twice the pages in flight
 
 struct WsLayout {
-    size_t err, tickets, part_ml, part_o, page_ml, logits, total;
+    size_t err, tickets, part_ml, part_o, page_lse, split_ml, logits, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -157,7 +157,8 @@ WsLayout ws_layout(const delta_desc* d, int batch, int max_pages, bool with_logi
     w.tickets = off;    off += align256(size_t(batch) * d->num_kv_heads * sizeof(int));
     w.part_ml = off;    off += align256(rows * S * sizeof(float2));
     w.part_o = off;     off += align256(rows * S * d->head_dim * sizeof(float));
-    w.page_ml = off;    off += align256(rows * size_t(max_pages) * sizeof(float2));
+    w.page_lse = off;   off += align256(rows * size_t(max_pages) * sizeof(float));
+    w.split_ml = off;   off += align256(rows * S * sizeof(float2));
     w.logits = off;     off += with_logits ? align256(rows * size_t(max_pages) * kPage * sizeof(float)) : 0;
     w.total = off;
     return w;
@@ -537,7 +538,8 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.mode = mode;
     prm.part_ml = reinterpret_cast<float2*>(base + L.part_ml);
     prm.part_o = reinterpret_cast<float*>(base + L.part_o);
-    prm.page_ml = reinterpret_cast<float2*>(base + L.page_ml);
+    prm.page_lse = reinterpret_cast<float*>(base + L.page_lse);
+    prm.split_ml = mode == kModeDelta ? reinterpret_cast<float2*>(base + L.split_ml) : nullptr;
     prm.err = reinterpret_cast<int*>(base + L.err);
     prm.o = o;
     prm.num_clusters = plan.clusters;
@@ -551,7 +553,9 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     SelectParams sp2{};
     sp2.indptr = pt->page_indptr;
     sp2.kv_len = pt->kv_len;
-    sp2.page_ml = prm.page_ml;
+    sp2.page_lse = prm.page_lse;
+    sp2.split_ml = prm.split_ml;
+    sp2.num_splits = S;
     sp2.num_q_heads = Hq;
     sp2.max_pages = pt->max_pages_per_seq;
     sp2.budget_pages = sp->budget_pages;
@@ -568,8 +572,10 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     int C = int((int64_t(Hq) * maxp + 16383) / 16384);
     C = C < 1 ? 1 : (C > 16 ? 16 : C);
     const int chunk = (maxp + C - 1) / C;
-    const SelectSmem SL{chunk, C, Hq};
-    const size_t smem_max = SelectSmem{kMaxSelectPages, 16, kMaxQHeadsSelect}.bytes();
+    const SelectSmem SL{chunk, C};
+    // C >= Hq * maxp / 16384 (or 16) keeps a CTA's pages at 16384 or fewer
+    if (chunk > kMaxSelectChunk) return DELTA_ERR_UNSUPPORTED;
+    const size_t smem_max = SelectSmem{kMaxSelectChunk, 16}.bytes();
     if (!configure_kernel(reinterpret_cast<const void*>(score_select_kernel), smem_max)) return DELTA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C, pt->batch);

@@ -9,7 +9,9 @@ namespace delta {
 struct SelectParams {
     const int32_t* indptr;
     const int32_t* kv_len;
-    const float2* page_ml;  // [B][Hq][max_pages]
+    const float* page_lse;   // [B][Hq][max_pages] log2-sum-exp of each page's base-2 logits
+    const float2* split_ml;  // [B][Hq][num_splits] (max, sum) of each decode split
+    int32_t num_splits;
     int32_t num_q_heads;
     int32_t max_pages;
     int32_t budget_pages, sink_tokens, recency_tokens;
@@ -55,23 +57,26 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& 
     return res;
 }
 
-// Shared-memory plan of the selection cluster (dynamic): keys of this CTA's pages, per-head
-// partial totals received from every CTA, double-buffered histograms received from every CTA.
+// Shared-memory plan of the selection cluster (dynamic): keys of this CTA's pages, the keys of the
+// threshold bucket (one-CTA path), double-buffered histograms and the compaction counts received
+// from every CTA.
 struct SelectSmem {
-    int chunk, C, Hq;
+    int chunk, C;
     __host__ __device__ size_t keys() const { return 0; }
-    __host__ __device__ size_t mz() const { return (size_t(chunk) * 4 + 15) & ~size_t(15); }
-    __host__ __device__ size_t hist() const { return mz() + size_t(C) * Hq * 8; }
+    __host__ __device__ size_t list() const { return (size_t(chunk) * 4 + 15) & ~size_t(15); }
+    __host__ __device__ size_t hist() const { return list() + ((size_t(chunk) * 4 + 15) & ~size_t(15)); }
     __host__ __device__ size_t counts() const { return hist() + size_t(2) * C * 256 * 4; }
     __host__ __device__ size_t bytes() const { return counts() + size_t(C) * 8; }
 };
 
 // One thread-block cluster per sequence; CTA r of C owns pages [r*chunk, (r+1)*chunk).
-// 1. per-head totals over the page partials, M_h = max_j m_hj and Z_h = sum_j 2^(m_hj - M_h) l_hj
-//    (each CTA over its pages, exchanged through distributed shared memory);
-// 2. page scores S_j = sum_h 2^(m_hj - M_h) l_hj / Z_h -> order-preserving keys;
-// 3. MSB-first 4 x 8-bit radix select of the k-th largest candidate key (histograms summed over
-//    the cluster), candidates being the pages neither sink nor recency;
+// 1. per-head normalisers c_h = log2 sum_j 2^(lse_hj), combined from the decode splits' (max, sum)
+//    states (a few per head, so every CTA does all heads and nothing is exchanged);
+// 2. page scores S_j = sum_h 2^(lse_hj - c_h) -> order-preserving keys;
+// 3. the k-th largest candidate key T (candidates: pages neither sink nor recency).  One CTA:
+//    a 256-bucket histogram over [min, max] of the keys, then the exact rank inside the bucket
+//    holding the k-th; a cluster: MSB-first 4 x 8-bit radix select with histograms summed over
+//    the cluster;
 // 4. ascending compaction of sink U recency U {key > T} U {the first (k - #greater) keys == T in
 //    page order} with cluster-wide offsets.
 // Every exchange pushes into the other CTAs' shared memory and is followed by one cluster barrier,
@@ -86,15 +91,17 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     };
     extern __shared__ __align__(16) unsigned char sm[];
     const int Hq = p.num_q_heads;
-    const SelectSmem L{chunk, C, Hq};
+    const SelectSmem L{chunk, C};
     uint32_t* keys = reinterpret_cast<uint32_t*>(sm + L.keys());
-    float2* recv_mz = reinterpret_cast<float2*>(sm + L.mz());        // [C][Hq]
+    uint32_t* blist = reinterpret_cast<uint32_t*>(sm + L.list());
     uint32_t* recv_hist = reinterpret_cast<uint32_t*>(sm + L.hist());  // [2][C][256]
     int2* recv_cnt = reinterpret_cast<int2*>(sm + L.counts());         // [C]
-    __shared__ float headM[kMaxQHeadsSelect], headZ[kMaxQHeadsSelect];
-    __shared__ uint32_t hist[256];
+    __shared__ float headC[kMaxQHeadsSelect];
+    __shared__ uint32_t hist[2][256];
     __shared__ int warp_sums[33];
-    __shared__ uint32_t s_digit, s_above;
+    __shared__ uint32_t s_digit[2], s_above[2];
+    __shared__ uint32_t s_kmin[32], s_kmax[32], s_T, s_need;
+    __shared__ int s_m;
 
     const int b = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -114,54 +121,54 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     const int k = p.budget_pages;
     const bool take_all = ncand <= k;
 
-    // 1. per-head partial totals over this CTA's pages (a warp per head), pushed to every CTA
+    const int sub = tid & 1;
+
+    // 1. per-head normaliser from the splits' states, a warp per head: the maximum first, then the
+    //    rescaled sum, so the exponentials are independent (no serial online update)
     for (int h = warp; h < Hq; h += kSelectThreads / 32) {
-        const float2* pm = p.page_ml + (size_t(b) * Hq + h) * p.max_pages;
+        const float2* ps = p.split_ml + (size_t(b) * Hq + h) * p.num_splits;
         float M = -INFINITY, Z = 0.f;
-        // sixteen independent loads in flight per lane, then an online (max, sum) update
-        for (int base = j0; base < j1; base += 32 * 16) {
+        for (int base = 0; base < p.num_splits; base += 32 * 16) {   // one round up to 512 splits
             float2 v[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                const int j = base + lane + 32 * u;
-                v[u] = (j < j1) ? pm[j] : make_float2(-INFINITY, 0.f);
+                const int s = base + lane + 32 * u;
+                v[u] = (s < p.num_splits) ? ps[s] : make_float2(-INFINITY, 0.f);
             }
+            float Mr = v[0].x;
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const float Mn = fmaxf(M, v[u].x);
-                const float mu = (Mn == -INFINITY) ? 0.f : Mn;
-                Z = Z * exp2_approx(M - mu) + v[u].y * exp2_approx(v[u].x - mu);
-                M = Mn;
-            }
-        }
+            for (int u = 1; u < 16; ++u) Mr = fmaxf(Mr, v[u].x);
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const float Mo = __shfl_xor_sync(0xffffffffu, M, o), Zo = __shfl_xor_sync(0xffffffffu, Z, o);
-            const float Mn = fmaxf(M, Mo);
+            for (int o = 16; o >= 1; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
+            const float Mn = fmaxf(M, Mr);
             const float mu = (Mn == -INFINITY) ? 0.f : Mn;
-            Z = Z * exp2_approx(M - mu) + Zo * exp2_approx(Mo - mu);
+            float z = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) z = fmaf(v[u].y, exp2_approx(v[u].x - mu), z);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            Z = Z * exp2_approx(M - mu) + z;
             M = Mn;
         }
-        if (lane < C) cluster.map_shared_rank(recv_mz, lane)[rank * Hq + h] = make_float2(M, Z);
+        // no token of the head: every page term is 2^(-inf) = 0
+        if (lane == 0) headC[h] = (Z > 0.f) ? M + log2_approx(Z) : INFINITY;
     }
-    cluster_barrier();
-    for (int h = tid; h < Hq; h += kSelectThreads) {
-        float M = -INFINITY, Z = 0.f;
-        for (int j = 0; j < C; ++j) {
-            const float2 v = recv_mz[j * Hq + h];
-            const float Mn = fmaxf(M, v.x);
-            const float mu = (Mn == -INFINITY) ? 0.f : Mn;
-            Z = Z * exp2_approx(M - mu) + v.y * exp2_approx(v.x - mu);
-            M = Mn;
-        }
-        headM[h] = M;
-        headZ[h] = 1.f / Z;   // stored as the reciprocal: the score pass multiplies
-    }
+    if (tid < 256) hist[0][tid] = 0;
     __syncthreads();
 
     // 2. page scores of this CTA's pages
+    uint32_t kmin_loc = 0xffffffffu, kmax_loc = 0u;
+    auto put_key = [&](int j, float sc) {
+        const uint32_t key = order_key(sc);
+        keys[j - j0] = key;
+        if (!forced(j)) {
+            kmin_loc = min(kmin_loc, key);
+            kmax_loc = max(kmax_loc, key);
+        }
+        if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
+    };
     if (p.logits != nullptr) {
-        // HEAD_MAX: S_j = sum over the page's tokens t < n of max_h 2^(s_ht - M_h) / Z_h.  A warp per
+        // HEAD_MAX: S_j = sum over the page's tokens t < n of max_h 2^(s_ht - c_h).  A warp per
         // page, lanes over heads, each lane holding the page's 16 token maxima of its heads.
         const size_t hs = size_t(p.max_pages) * kPage;
         for (int j = j0 + warp; j < j1; j += kSelectThreads / 32) {
@@ -170,14 +177,14 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
             for (int t = 0; t < kPage; ++t) mx[t] = 0.f;
             for (int h = lane; h < Hq; h += 32) {
                 const float4* lg = reinterpret_cast<const float4*>(p.logits + (size_t(b) * Hq + h) * hs + size_t(j) * kPage);
-                const float inv = headZ[h];
+                const float c = headC[h];
 #pragma unroll
                 for (int q4 = 0; q4 < kPage / 4; ++q4) {
                     const float4 v = lg[q4];
-                    mx[4 * q4 + 0] = fmaxf(mx[4 * q4 + 0], exp2_approx(v.x - headM[h]) * inv);
-                    mx[4 * q4 + 1] = fmaxf(mx[4 * q4 + 1], exp2_approx(v.y - headM[h]) * inv);
-                    mx[4 * q4 + 2] = fmaxf(mx[4 * q4 + 2], exp2_approx(v.z - headM[h]) * inv);
-                    mx[4 * q4 + 3] = fmaxf(mx[4 * q4 + 3], exp2_approx(v.w - headM[h]) * inv);
+                    mx[4 * q4 + 0] = fmaxf(mx[4 * q4 + 0], exp2_approx(v.x - c));
+                    mx[4 * q4 + 1] = fmaxf(mx[4 * q4 + 1], exp2_approx(v.y - c));
+                    mx[4 * q4 + 2] = fmaxf(mx[4 * q4 + 2], exp2_approx(v.z - c));
+                    mx[4 * q4 + 3] = fmaxf(mx[4 * q4 + 3], exp2_approx(v.w - c));
                 }
             }
             float sc = 0.f;
@@ -188,65 +195,146 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
                 for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
                 if (j * kPage + t < n) sc += v;
             }
-            if (lane == 0) {
-                keys[j - j0] = order_key(sc);
-                if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
-            }
+            if (lane == 0) put_key(j, sc);
         }
     } else {
         // HEAD_SUM: two threads per page, each summing every other head with up to sixteen
-        // independent loads in flight, so a page's partials arrive in one round
-        const int sub = tid & 1;
+        // independent loads in flight, so a page's terms arrive in one round
         for (int base = j0; base < j1; base += kSelectThreads / 2) {   // uniform trip count
             const int j = base + (tid >> 1);
             const bool active = j < j1;
-            const float2* pm = p.page_ml + size_t(b) * Hq * p.max_pages + (active ? j : j0);
+            const float* pl = p.page_lse + size_t(b) * Hq * p.max_pages + (active ? j : j0);
             float sc = 0.f;
             for (int hb = 0; hb < Hq; hb += 32) {
-                float2 v[16];
+                float v[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int h = hb + sub + 2 * u;
-                    v[u] = (active && h < Hq) ? pm[size_t(h) * p.max_pages] : make_float2(-INFINITY, 0.f);
+                    v[u] = (active && h < Hq) ? pl[size_t(h) * p.max_pages] : -INFINITY;
                 }
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int h = hb + sub + 2 * u;
-                    if (h < Hq) sc += exp2_approx(v[u].x - headM[h]) * v[u].y * headZ[h];
+                    if (h < Hq) sc += exp2_approx(v[u] - headC[h]);
                 }
             }
             sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-            if (active && sub == 0) {
-                keys[j - j0] = order_key(sc);
-                if (p.page_scores != nullptr) p.page_scores[size_t(b) * p.max_pages + j] = sc;
-            }
+            if (active && sub == 0) put_key(j, sc);
         }
     }
+    // range of the candidate keys (the one-CTA threshold search buckets it), per warp here and
+    // over the CTA after the barrier
+    kmin_loc = __reduce_min_sync(0xffffffffu, kmin_loc);
+    kmax_loc = __reduce_max_sync(0xffffffffu, kmax_loc);
+    if (lane == 0) {
+        s_kmin[warp] = kmin_loc;
+        s_kmax[warp] = kmax_loc;
+    }
+    if (tid == 0) s_m = 0;
     __syncthreads();
 
-    // 3. radix select of the k-th largest candidate key over the whole cluster
+    // 3. radix select of the k-th largest candidate key over the whole cluster.  Histograms and
+    //    the chosen digit are double-buffered, so a pass needs two block barriers.
     uint32_t T = 0, need_eq = 0;
-    if (!take_all && k > 0) {
+    if (!take_all && k > 0 && C == 1) {
+        // one CTA: bucket b(key) = (key - kmin) >> sh in [0, 255] (monotone in the key)
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll 8
+        for (int w = 0; w < kSelectThreads / 32; ++w) {
+            kmin = min(kmin, s_kmin[w]);
+            kmax = max(kmax, s_kmax[w]);
+        }
+        const uint32_t span = kmax - kmin;   // ncand > k >= 1 candidates: kmin <= kmax
+        const int sh = max(0, 24 - __clz(span));
+        // warp-aggregated: most keys crowd into a few buckets, so lanes of one bucket add once
+        for (int base = j0; base < j1; base += kSelectThreads) {   // uniform trip count
+            const int j = base + tid;
+            const uint32_t bk = (j < j1 && !forced(j)) ? (keys[j - j0] - kmin) >> sh : 0xffffffffu;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bk);
+            if (bk != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[0][bk], uint32_t(__popc(peers)));
+        }
+        __syncthreads();
+        if (tid < 32) {   // the bucket holding the k-th largest, and the keys in higher buckets
+            uint32_t c[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { c[i] = hist[0][255 - 8 * tid - i]; sum += c[i]; }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += y;
+            }
+            const uint32_t excl = incl - sum;
+            if (excl < uint32_t(k) && uint32_t(k) <= incl) {
+                uint32_t above = excl;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (above + c[i] >= uint32_t(k)) { s_digit[0] = 255 - 8 * tid - i; s_above[0] = above; break; }
+                    above += c[i];
+                }
+            }
+        }
+        __syncthreads();
+        const uint32_t tb = s_digit[0];
+        const int kk = k - int(s_above[0]);   // rank of T inside its bucket, 1-based
+        // gather the bucket's keys (warp-aggregated slots; uniform trip count for the ballot)
+        for (int base = j0; base < j1; base += kSelectThreads) {
+            const int j = base + tid;
+            const bool in = j < j1 && !forced(j) && ((keys[j - j0] - kmin) >> sh) == tb;
+            const uint32_t bal = __ballot_sync(0xffffffffu, in);
+            int slot = 0;
+            if (lane == 0 && bal != 0u) slot = atomicAdd(&s_m, __popc(bal));
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+            if (in) blist[slot + __popc(bal & ((1u << lane) - 1u))] = keys[j - j0];
+        }
+        __syncthreads();
+        // T = the key v of the bucket with #(> v) < kk <= #(>= v); every holder of v writes the same
+        const int m = s_m;
+        for (int i = tid; i < m; i += kSelectThreads) {
+            const uint32_t v = blist[i];
+            int gt = 0, ge = 0;
+            for (int t = 0; t < m; ++t) {
+                const uint32_t w = blist[t];
+                gt += w > v ? 1 : 0;
+                ge += w >= v ? 1 : 0;
+            }
+            if (gt < kk && kk <= ge) {
+                s_T = v;
+                s_need = uint32_t(kk - gt);
+            }
+        }
+        __syncthreads();
+        T = s_T;
+        need_eq = s_need;   // how many of the keys equal to T are taken (lowest page indices first)
+    } else if (!take_all && k > 0) {
         uint32_t prefix = 0, mask = 0, kk = k;
         for (int pass = 0, shift = 24; shift >= 0; ++pass, shift -= 8) {
-            for (int i = tid; i < 256; i += kSelectThreads) hist[i] = 0;
-            __syncthreads();
-            for (int j = j0 + tid; j < j1; j += kSelectThreads) {
-                const uint32_t key = keys[j - j0];
-                if (!forced(j) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            const int cur = pass & 1;
+            // warp-aggregated: the leading digits of most keys agree, so lanes with equal digits
+            // add once (uniform trip count for the warp-wide match)
+            for (int base = j0; base < j1; base += kSelectThreads) {
+                const int j = base + tid;
+                uint32_t dig = 0xffffffffu;
+                if (j < j1 && !forced(j)) {
+                    const uint32_t key = keys[j - j0];
+                    if ((key & mask) == prefix) dig = (key >> shift) & 255u;
+                }
+                const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+                if (dig != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[cur][dig], uint32_t(__popc(peers)));
             }
+            if (tid < 256) hist[cur ^ 1][tid] = 0;   // the next pass's buffer (last read two barriers ago)
             __syncthreads();
             if (C > 1) {   // sum the histograms of the cluster (one CTA: already the total)
-                uint32_t* rh = recv_hist + (pass & 1) * C * 256;
+                uint32_t* rh = recv_hist + cur * C * 256;
                 for (int i = tid; i < C * 256; i += kSelectThreads) {
                     const int j = i >> 8, bin = i & 255;
-                    cluster.map_shared_rank(rh, j)[rank * 256 + bin] = hist[bin];
+                    cluster.map_shared_rank(rh, j)[rank * 256 + bin] = hist[cur][bin];
                 }
                 cluster_barrier();
                 if (tid < 256) {
                     uint32_t t = 0;
                     for (int j = 0; j < C; ++j) t += rh[j * 256 + tid];
-                    hist[tid] = t;
+                    hist[cur][tid] = t;
                 }
                 __syncthreads();
             }
@@ -254,7 +342,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
                 // lane covers digits 255-8*lane .. 248-8*lane (descending)
                 uint32_t c[8], sum = 0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * tid - i]; sum += c[i]; }
+                for (int i = 0; i < 8; ++i) { c[i] = hist[cur][255 - 8 * tid - i]; sum += c[i]; }
                 uint32_t incl = sum;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -266,37 +354,38 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
                     uint32_t above = excl;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        if (above + c[i] >= kk) { s_digit = 255 - 8 * tid - i; s_above = above; break; }
+                        if (above + c[i] >= kk) { s_digit[cur] = 255 - 8 * tid - i; s_above[cur] = above; break; }
                         above += c[i];
                     }
                 }
             }
             __syncthreads();
-            prefix |= s_digit << shift;
+            prefix |= s_digit[cur] << shift;
             mask |= 0xffu << shift;
-            kk -= s_above;
-            __syncthreads();
+            kk -= s_above[cur];
         }
         T = prefix;
         need_eq = kk;   // how many of the keys equal to T are taken (lowest page indices first)
     }
 
-    // 4. cluster-wide offsets, then the ascending compaction of this CTA's pages
+    // 4. cluster-wide offsets, then the ascending compaction of this CTA's pages.  Pages equal to T
+    //    are taken in page order, so the taken ones before a thread follow from the equal ones
+    //    before it: one (packed) scan gives every thread its output position.
     const int per = (nloc + kSelectThreads - 1) / kSelectThreads;
     const int jb = j0 + tid * per, je = min(jb + per, j1);
     const bool radix = !take_all && k > 0;
     int eq_cnt = 0, gtf_cnt = 0;
     for (int j = jb; j < je; ++j) {
-        if (forced(j)) { ++gtf_cnt; continue; }
-        if (take_all) { ++gtf_cnt; continue; }
+        if (forced(j) || take_all) { ++gtf_cnt; continue; }
         if (!radix) continue;
         const uint32_t key = keys[j - j0];
         if (key > T) ++gtf_cnt;
         else if (key == T) ++eq_cnt;
     }
-    int eq_tot_loc, gtf_tot_loc;
-    const int eq_rank_loc = block_exclusive_scan(eq_cnt, warp_sums, eq_tot_loc);
-    block_exclusive_scan(gtf_cnt, warp_sums, gtf_tot_loc);
+    int tot_loc;   // both counts fit 15 bits: a CTA owns at most 16384 pages
+    const int packed = block_exclusive_scan(eq_cnt | (gtf_cnt << 16), warp_sums, tot_loc);
+    const int eq_rank_loc = packed & 0xffff, gtf_rank_loc = packed >> 16;
+    const int eq_tot_loc = tot_loc & 0xffff, gtf_tot_loc = tot_loc >> 16;
     if (tid < C) cluster.map_shared_rank(recv_cnt, tid)[rank] = make_int2(eq_tot_loc, gtf_tot_loc);
     cluster_barrier();
     int eq_cum = 0, eq_before = 0, sel_before = 0, total = 0;
@@ -310,21 +399,20 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
         total += v.y + taken;
         eq_cum += v.x;
     }
-    auto selected = [&](int j, int& eq_seen) -> bool {
-        if (forced(j) || take_all) return true;
-        if (!radix) return false;
-        const uint32_t key = keys[j - j0];
-        if (key > T) return true;
-        if (key == T) return uint32_t(eq_before + eq_rank_loc + eq_seen++) < need_eq;
-        return false;
-    };
-    int cnt = 0, seen = 0;
-    for (int j = jb; j < je; ++j) cnt += selected(j, seen) ? 1 : 0;
-    int local_total;
-    int pos = sel_before + block_exclusive_scan(cnt, warp_sums, local_total);
-    seen = 0;
+    const int eq_left = max(int(need_eq) - eq_before, 0);            // T-valued pages this CTA may still take
+    int pos = sel_before + gtf_rank_loc + min(eq_left, eq_rank_loc);
+    int eq_seen = eq_rank_loc;
     for (int j = jb; j < je; ++j) {
-        if (selected(j, seen)) {
+        bool take;
+        if (forced(j) || take_all) {
+            take = true;
+        } else if (!radix) {
+            take = false;
+        } else {
+            const uint32_t key = keys[j - j0];
+            take = key > T || (key == T && eq_seen++ < eq_left);
+        }
+        if (take) {
             if (pos < p.sel_stride) p.sel_pages[size_t(b) * p.sel_stride + pos] = j;
             ++pos;
         }

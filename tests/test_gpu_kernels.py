@@ -198,11 +198,12 @@ def test_select_attn_matches_oracle(L, mode, G, Hkv, D, dtype, ctx, k, sink, rec
         assert ok, f"b={b}: gpu {gsel} vs oracle {ref_sel}"
 
 
-def test_select_exact_ties_across_cluster_ctas(L):
+@pytest.mark.parametrize("n,k,one_cta", [(16384 + 5, 700, False), (3000 + 5, 40, True)])
+def test_select_exact_ties(L, n, k, one_cta):
     # Identical keys give identical page scores: the selection must take the lowest-index
-    # candidates, and with 32 query heads x 1025 pages the selection runs as a 3-CTA cluster
-    # whose chunk boundaries fall inside the selected range.
-    n, k = 16384 + 5, 700
+    # candidates.  With 32 query heads x 1025 pages the selection runs as a 3-CTA cluster whose
+    # chunk boundaries fall inside the selected range; with 188 pages it runs in one CTA, where
+    # every candidate lands in the same threshold bucket.
     cfg = make_cfg(8, 4, 128, "bf16", [n], budget_pages=k, sink=16, rec=256)
     dc = device_case(cfg)
     dc.k_pools[0].fill_(1.0)
@@ -211,7 +212,7 @@ def test_select_exact_ties_across_cluster_ctas(L):
     sp = L.DeltaSelectParams(k, 16, 256, L.DELTA_HEAD_SUM)
     stride = L.sel_capacity(sp)
     maxp = dc.case.max_pages_per_seq
-    assert 32 * maxp > 2 * 16384
+    assert (32 * maxp <= 16384) == one_cta
     sel_cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
     sel_pages = torch.full((1, stride), -1, dtype=torch.int32, device="cuda")
     scores = torch.zeros((1, maxp), dtype=torch.float32, device="cuda")
