@@ -312,10 +312,10 @@ __device__ __forceinline__ void seq_count(const P& p, int b, SeqExtent& ex) {
 template <int D>
 constexpr int recv_floats() { return 4 + kMaxGroup * D + 16 * 4 + 16 * kMaxGroup * 2 + kMaxGroup * 2; }
 
-// Kernel prologue of the cluster merge, all threads, before any page work: thread 0 initialises
-// this CTA's receive barrier, then every thread arrives (relaxed) on the cluster barrier that the
-// epilogue waits on before its first remote store, so no CTA signals a barrier that its owner has
-// not initialised yet.  The wait is long satisfied when the epilogue reaches it.
+// Kernel prologue of the cluster merge, all threads, before the wait for the previous kernel:
+// thread 0 initialises this CTA's receive barrier, then one cluster barrier makes every CTA's
+// initialisation visible before any CTA can signal it (the CTAs of a cluster start together, so
+// this costs nothing while the previous kernel is still running).
 __device__ __forceinline__ void merge_prologue(float* recv) {
     if (threadIdx.x == 0) {
         mbar_init(reinterpret_cast<uint64_t*>(recv), 1);
@@ -323,6 +323,7 @@ __device__ __forceinline__ void merge_prologue(float* recv) {
     }
     __syncwarp();
     cluster_arrive_relaxed();
+    cluster_wait();
 }
 
 template <typename T, int D, int G, int NPART>
@@ -382,7 +383,6 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
         }
     }
     __syncthreads();
-    cluster_wait();   // every CTA of the cluster has initialised its receive barrier
     if (tid < C * G) {   // this CTA's (max, sum) of head h to cluster rank j
         const int j = tid / G, h = tid % G;
         st_async(cluster_addr(recv_ml + (rank * G + h) * 2, j), make_float2(cml[2 * h], cml[2 * h + 1]),

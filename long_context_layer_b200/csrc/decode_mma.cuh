@@ -192,13 +192,17 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     }
 
     if (p.mode == kModeSparse) {
+        // The selection's entries at the speculated positions are loaded together with its count
+        // (one round trip); they are the real ones whenever the count is the speculated one.
+        const int lp_real = (lane < nk_spec)
+                                ? p.sel_pages[size_t(b) * p.sel_stride + split * p.items_per_split + warp + lane * kWarps]
+                                : -1;
         seq_count(p, b, ex);
         i0 = split * p.items_per_split;
         const int i1 = min(i0 + p.items_per_split, ex.count);
         nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;
         // The speculation holds if the selection's logical pages of this warp's first chunk are the
         // ones guessed (the page table does not change within the step) and were all valid.
-        const int lp_real = (lane < nk) ? p.sel_pages[size_t(b) * p.sel_stride + i0 + warp + lane * kWarps] : -1;
         const bool all_same = __all_sync(0xffffffffu, lane >= nk || (lp_real == spec.lp_a && spec.ph_a >= 0)) &&
                               nk == nk_spec;
         if (all_same) {
