@@ -326,10 +326,13 @@ __device__ __forceinline__ void merge_prologue(float* recv) {
     cluster_wait();
 }
 
+// Part rr's records: outputs mo[rr * ostride + h * D + d], states ml[rr * mstride + 2 * h] (max,
+// sum) of base-2 logits; dml (delta-layers, same strides as ml) holds the states over the exact
+// fp32 page terms when those differ from ml.
 template <typename T, int D, int G, int NPART>
 __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
-                                               const float* mml, float* recv, int b, int g,
-                                               const float* dml = nullptr) {
+                                               const float* mml, float* recv, int b, int g, int ostride,
+                                               int mstride, const float* dml = nullptr) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = int(cluster.num_blocks());
@@ -345,58 +348,51 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
     // 1. this CTA's NPART states -> one state, pushed straight into the shared memory of the
     //    cluster CTA that owns each output element with asynchronous remote stores; each owner
     //    waits on its own barrier for the bytes of all C CTAs (no cluster-wide barrier, no round
-    //    trip).  Slices are multiples of 4 elements so every push is one 16-byte store.
+    //    trip).  Every thread combines the parts' states it needs itself (no barrier).  Slices
+    //    are multiples of 4 elements so every push is one 16-byte store.
     const int total = G * D;
     const int chunk = (((total + C - 1) / C) + 3) & ~3;
     uint64_t* rbar = reinterpret_cast<uint64_t*>(recv);
     recv += 4;
     float* recv_ml = recv + C * chunk;                                             // [C][G][2]
-    float* cml = recv_ml + C * G * 2;                                              // [G][2] this CTA
     const int e0 = rank * chunk, e1 = min(e0 + chunk, total);                      // this CTA's slice
     if (tid == 0) mbar_expect_tx(rbar, uint32_t(C) * (uint32_t(max(e1 - e0, 0)) * 4u + uint32_t(G) * 8u));
-    if (tid < G) {
+    auto part_max = [&](const float* ml, int h) {
         float M = -INFINITY;
 #pragma unroll
-        for (int rr = 0; rr < NPART; ++rr) M = fmaxf(M, mml[(rr * kMaxGroup + tid) * 2]);
+        for (int rr = 0; rr < NPART; ++rr) M = fmaxf(M, ml[rr * mstride + 2 * h]);
+        return M;
+    };
+    auto part_sum = [&](const float* ml, int h, float M) {
         const float mu = (M == -INFINITY) ? 0.f : M;
         float L = 0.f;
 #pragma unroll
-        for (int rr = 0; rr < NPART; ++rr)
-            L = fmaf(exp2_approx(mml[(rr * kMaxGroup + tid) * 2] - mu), mml[(rr * kMaxGroup + tid) * 2 + 1], L);
-        cml[2 * tid] = M;
-        cml[2 * tid + 1] = L;
-        if (p.split_ml != nullptr) {
-            // the selection's per-head totals are combined from these; dml (when given) holds the
-            // parts' states over the exact page terms
-            float Md = M, Ld = L;
-            if (dml != nullptr) {
-                Md = -INFINITY;
-#pragma unroll
-                for (int rr = 0; rr < NPART; ++rr) Md = fmaxf(Md, dml[(rr * kMaxGroup + tid) * 2]);
-                const float md = (Md == -INFINITY) ? 0.f : Md;
-                Ld = 0.f;
-#pragma unroll
-                for (int rr = 0; rr < NPART; ++rr)
-                    Ld = fmaf(exp2_approx(dml[(rr * kMaxGroup + tid) * 2] - md), dml[(rr * kMaxGroup + tid) * 2 + 1], Ld);
-            }
-            p.split_ml[(size_t(b) * Hq + h0 + tid) * p.num_splits + blockIdx.x] = make_float2(Md, Ld);
-        }
-    }
-    __syncthreads();
+        for (int rr = 0; rr < NPART; ++rr) L = fmaf(exp2_approx(ml[rr * mstride + 2 * h] - mu), ml[rr * mstride + 2 * h + 1], L);
+        return L;
+    };
     if (tid < C * G) {   // this CTA's (max, sum) of head h to cluster rank j
         const int j = tid / G, h = tid % G;
-        st_async(cluster_addr(recv_ml + (rank * G + h) * 2, j), make_float2(cml[2 * h], cml[2 * h + 1]),
-                 cluster_addr(rbar, j));
+        const float M = part_max(mml, h);
+        const float L = part_sum(mml, h, M);
+        st_async(cluster_addr(recv_ml + (rank * G + h) * 2, j), make_float2(M, L), cluster_addr(rbar, j));
+        if (j == 0 && p.split_ml != nullptr) {   // the selection combines its per-head totals from these
+            float Md = M, Ld = L;
+            if (dml != nullptr) {
+                Md = part_max(dml, h);
+                Ld = part_sum(dml, h, Md);
+            }
+            p.split_ml[(size_t(b) * Hq + h0 + h) * p.num_splits + blockIdx.x] = make_float2(Md, Ld);
+        }
     }
     for (int q4 = tid; q4 * 4 < total; q4 += nthr) {
         const int idx = q4 * 4, h = idx / D, d = idx % D;    // D is a multiple of 4: one head per group
-        const float M = cml[2 * h];
+        const float M = part_max(mml, h);
         const float mu = (M == -INFINITY) ? 0.f : M;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int rr = 0; rr < NPART; ++rr) {
-            const float w = exp2_approx(mml[(rr * kMaxGroup + h) * 2] - mu);
-            const float4 v = *reinterpret_cast<const float4*>(&mo[(rr * kMaxGroup + h) * D + d]);
+            const float w = exp2_approx(mml[rr * mstride + 2 * h] - mu);
+            const float4 v = *reinterpret_cast<const float4*>(&mo[rr * ostride + h * D + d]);
             acc.x = fmaf(w, v.x, acc.x);
             acc.y = fmaf(w, v.y, acc.y);
             acc.z = fmaf(w, v.z, acc.z);

@@ -64,8 +64,9 @@ struct MmaSmem {
     static constexpr uint32_t kBox = 16 * 128;                // one box: 16 rows x 128 bytes
     static constexpr uint32_t kPage = 2 * kBoxes * kBox;      // K and V of one page, one KV head
     static constexpr size_t kStages = size_t(kWarps) * STAGES * kPage;
-    static constexpr size_t kMerge = size_t(kWarps + 1) * kMaxGroup * (D + 2) * sizeof(float);
-    static constexpr size_t kMain = kStages > kMerge ? kStages : kMerge;
+    // each warp's merge record ([8][D] outputs, two [8][2] states) reuses its own stages
+    static_assert(size_t(STAGES) * kPage >= (size_t(kMaxGroup) * D + 4 * kMaxGroup) * sizeof(float), "merge record");
+    static constexpr size_t kMain = kStages;
     static constexpr size_t kBars = size_t(kWarps) * STAGES * sizeof(uint64_t);
     static constexpr size_t kRecv = size_t(recv_floats<D>()) * sizeof(float);
     // the page-table row of the sequence, staged for sparse layers (deep variant only: the
@@ -415,33 +416,37 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         for (int k = consumed + 1; k < min(consumed + STAGES, nk); ++k) mbar_wait(&wbar[k % STAGES], parity(k));
     }
 
-    // ---- merge the 4 warps' states of this CTA, then the splits
-    __syncthreads();
-    float* mo = reinterpret_cast<float*>(smem);          // [4][8][D]
-    float* mml = mo + kWarps * kMaxGroup * D;            // [4][8][2]
+    // ---- this warp's state into its own stage area (all of its copies have landed and no other
+    // warp touches that area), one barrier, then the merge of the 4 warps and of the splits
+    __syncwarp();
+    float* po = reinterpret_cast<float*>(wst);           // [8][D] outputs
+    float* pml = po + kMaxGroup * D;                      // [8][2] (max, sum)
+    float* pdl = pml + kMaxGroup * 2;                     // [8][2] delta-layers: over the fp32 page terms
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) {
         const int d = mt * 16 + g4;
-        mo[(warp * kMaxGroup + 2 * t4) * D + d] = acc[mt][0];
-        mo[(warp * kMaxGroup + 2 * t4 + 1) * D + d] = acc[mt][1];
-        mo[(warp * kMaxGroup + 2 * t4) * D + d + 8] = acc[mt][2];
-        mo[(warp * kMaxGroup + 2 * t4 + 1) * D + d + 8] = acc[mt][3];
+        po[(2 * t4) * D + d] = acc[mt][0];
+        po[(2 * t4 + 1) * D + d] = acc[mt][1];
+        po[(2 * t4) * D + d + 8] = acc[mt][2];
+        po[(2 * t4 + 1) * D + d + 8] = acc[mt][3];
     }
-    float* dml = mml + kWarps * kMaxGroup * 2;           // [4][8][2] delta-layers
     if (g4 == 0) {
-        mml[(warp * kMaxGroup + 2 * t4) * 2 + 0] = m_run[0];
-        mml[(warp * kMaxGroup + 2 * t4) * 2 + 1] = l_run[0];
-        mml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 0] = m_run[1];
-        mml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 1] = l_run[1];
+        pml[(2 * t4) * 2 + 0] = m_run[0];
+        pml[(2 * t4) * 2 + 1] = l_run[0];
+        pml[(2 * t4 + 1) * 2 + 0] = m_run[1];
+        pml[(2 * t4 + 1) * 2 + 1] = l_run[1];
         if (p.mode == kModeDelta) {
-            dml[(warp * kMaxGroup + 2 * t4) * 2 + 0] = dm_run[0];
-            dml[(warp * kMaxGroup + 2 * t4) * 2 + 1] = dl_run[0];
-            dml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 0] = dm_run[1];
-            dml[(warp * kMaxGroup + 2 * t4 + 1) * 2 + 1] = dl_run[1];
+            pdl[(2 * t4) * 2 + 0] = dm_run[0];
+            pdl[(2 * t4) * 2 + 1] = dl_run[0];
+            pdl[(2 * t4 + 1) * 2 + 0] = dm_run[1];
+            pdl[(2 * t4 + 1) * 2 + 1] = dl_run[1];
         }
     }
     __syncthreads();
-    merge_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo, mml, recv, b, g, dml);
+    constexpr int kPart = STAGES * int(S::kPage) / 4;     // floats between two warps' records
+    const float* mo0 = reinterpret_cast<const float*>(smem);
+    merge_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo0, mo0 + kMaxGroup * D, recv, b, g, kPart, kPart,
+                                                (p.mode == kModeDelta) ? mo0 + kMaxGroup * D + kMaxGroup * 2 : nullptr);
 }
 
 }  // namespace delta

@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         mml[(r * kMaxGroup + hl) * 2 + 1] = l_run;
     }
     __syncthreads();
-    merge_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, recv, b, g);
+    merge_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, recv, b, g, kMaxGroup * D, kMaxGroup * 2);
 }
 
 }  // namespace delta
