@@ -349,7 +349,12 @@ SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) 
         per_cluster = (e != nullptr && atoi(e) > 0) ? atoi(e) : 256;
     }
     // Up to 512 pages per (sequence, KV head) one cluster is faster (measured on the 8k stack).
-    const int max_clusters = (items <= 512 || items / per_cluster < 1) ? 1 : items / per_cluster;
+    static int one_cluster = -1;
+    if (one_cluster < 0) {
+        const char* e = getenv("DELTA_ONE_CLUSTER_PAGES");   // tuning override for sweeps
+        one_cluster = (e != nullptr && atoi(e) >= 0) ? atoi(e) : 512;
+    }
+    const int max_clusters = (items <= one_cluster || items / per_cluster < 1) ? 1 : items / per_cluster;
     SplitPlan best = pl;
     int best_ctas = -1;
     for (int c = pl.cluster; c >= 1; --c) {
