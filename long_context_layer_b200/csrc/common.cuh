@@ -224,14 +224,15 @@ struct SeqExtent {
 };
 
 // QUIET: a speculative lookup (before the wait, for an L2 prefetch only) that raises no flags.
-template <bool QUIET = false, typename P>
+// W: warps of the CTA (warp w streams items i0 + w, i0 + w + W, ...).
+template <bool QUIET = false, int W = kWarps, typename P>
 __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int b, int i0, int warp, int nk, int kbase,
                                             int lane, int& lp, int& ph) {
     const int k = kbase + lane;
     lp = -1;
     ph = -1;
     if (k >= nk) return;
-    const int i = i0 + warp + k * kWarps;
+    const int i = i0 + warp + k * W;
     lp = (p.mode == kModeSparse) ? p.sel_pages[size_t(b) * p.sel_stride + i] : i;
     if (lp < 0 || lp >= ex.N) {
         if (!QUIET) atomicOr(p.err, kErrSel);
@@ -246,23 +247,23 @@ __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int
     ph = int(x);
 }
 
-template <typename P>
+template <int W = kWarps, typename P>
 __device__ __forceinline__ void pages_init(WarpPages& w, const P& p, const SeqExtent& ex, int b, int i0, int warp,
                                            int nk, int lane) {
     w.cur = 0;
-    fetch_pages(p, ex, b, i0, warp, nk, 0, lane, w.lp_a, w.ph_a);
-    fetch_pages(p, ex, b, i0, warp, nk, 32, lane, w.lp_b, w.ph_b);
+    fetch_pages<false, W>(p, ex, b, i0, warp, nk, 0, lane, w.lp_a, w.ph_a);
+    fetch_pages<false, W>(p, ex, b, i0, warp, nk, 32, lane, w.lp_b, w.ph_b);
 }
 
 // Called by all lanes at the top of iteration k (uniform).
-template <typename P>
+template <int W = kWarps, typename P>
 __device__ __forceinline__ void pages_advance(WarpPages& w, const P& p, const SeqExtent& ex, int b, int i0, int warp,
                                               int nk, int lane, int k) {
     if (k > 0 && (k & 31) == 0) {
         w.cur = k >> 5;
         w.lp_a = w.lp_b;
         w.ph_a = w.ph_b;
-        fetch_pages(p, ex, b, i0, warp, nk, (w.cur + 1) * 32, lane, w.lp_b, w.ph_b);
+        fetch_pages<false, W>(p, ex, b, i0, warp, nk, (w.cur + 1) * 32, lane, w.lp_b, w.ph_b);
     }
 }
 
@@ -329,7 +330,7 @@ __device__ __forceinline__ void merge_prologue(float* recv) {
 // Part rr's records: outputs mo[rr * ostride + h * D + d], states ml[rr * mstride + 2 * h] (max,
 // sum) of base-2 logits; dml (delta-layers, same strides as ml) holds the states over the exact
 // fp32 page terms when those differ from ml.
-template <typename T, int D, int G, int NPART>
+template <typename T, int D, int G, int NPART, int NTHR = kThreads>
 __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
                                                const float* mml, float* recv, int b, int g, int ostride,
                                                int mstride, const float* dml = nullptr) {
@@ -466,7 +467,7 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
         sml[idx] = (M == -INFINITY) ? 0.f : exp2_approx(sml[idx] - M) / Ls;
     }
     __syncthreads();
-    constexpr int J = (G * D + kThreads - 1) / kThreads;   // outputs per thread
+    constexpr int J = (G * D + NTHR - 1) / NTHR;   // outputs per thread
     float a[J];
 #pragma unroll
     for (int j = 0; j < J; ++j) a[j] = 0.f;
@@ -474,7 +475,7 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
     for (int c = 0; c < nC; ++c) {
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-            const int idx = tid + j * kThreads;
+            const int idx = tid + j * NTHR;
             if (idx < G * D) {
                 const int h = idx / D, d = idx % D;
                 a[j] = fmaf(sml[h * nC + c], __ldcg(p.part_o + ((size_t(b) * Hq + h0 + h) * nC + c) * D + d), a[j]);
@@ -483,7 +484,7 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
     }
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-        const int idx = tid + j * kThreads;
+        const int idx = tid + j * NTHR;
         if (idx < G * D) out[(size_t(b) * Hq + h0 + idx / D) * D + idx % D] = Elem<T>::from_f(a[j]);
     }
 }

@@ -58,35 +58,31 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // Shared-memory plan of the tensor-core kernel.
-template <int D, int STAGES>
+template <int D, int STAGES, int WARPS = kWarps>
 struct MmaSmem {
     static constexpr int kBoxes = D / 64;                     // 64-column (128-byte) boxes per row
     static constexpr uint32_t kBox = 16 * 128;                // one box: 16 rows x 128 bytes
     static constexpr uint32_t kPage = 2 * kBoxes * kBox;      // K and V of one page, one KV head
-    static constexpr size_t kStages = size_t(kWarps) * STAGES * kPage;
+    static constexpr size_t kStages = size_t(WARPS) * STAGES * kPage;
     // each warp's merge record ([8][D] outputs, two [8][2] states) reuses its own stages
     static_assert(size_t(STAGES) * kPage >= (size_t(kMaxGroup) * D + 4 * kMaxGroup) * sizeof(float), "merge record");
     static constexpr size_t kMain = kStages;
-    static constexpr size_t kBars = size_t(kWarps) * STAGES * sizeof(uint64_t);
+    static constexpr size_t kBars = size_t(WARPS) * STAGES * sizeof(uint64_t);
     static constexpr size_t kRecv = size_t(recv_floats<D>()) * sizeof(float);
-    // the page-table row of the sequence, staged for sparse layers (deep variant only: the
-    // shallow one must keep two CTAs per SM)
-    static constexpr int kTable = STAGES >= 6 ? 4096 : 0;
-    static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kRecv + size_t(kTable) * 4;
+    static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kRecv;
 };
 
-template <int D, int G, int STAGES>
-__global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams p,
+template <int D, int G, int STAGES, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodeParams p,
                                                               const __grid_constant__ CUtensorMap tmap_k,
                                                               const __grid_constant__ CUtensorMap tmap_v) {
-    using S = MmaSmem<D, STAGES>;
+    using S = MmaSmem<D, STAGES, WARPS>;
     constexpr int KS = D / 16;   // k-steps of the QK product = M-tiles of the PV product
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem =
         smem_raw + ((1024 - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kMain);
     float* recv = reinterpret_cast<float*>(smem + S::kMain + S::kBars);
-    int32_t* table = reinterpret_cast<int32_t*>(smem + S::kMain + S::kBars + S::kRecv);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g4 = lane >> 2, t4 = lane & 3;
@@ -115,8 +111,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         seq_count(p, b, ex);
         i0 = split * p.items_per_split;
         const int i1 = min(i0 + p.items_per_split, ex.count);
-        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
-        pages_init(pages, p, ex, b, i0, warp, nk, lane);
+        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + WARPS - 1) / WARPS : 0;   // pages of this warp
+        pages_init<WARPS>(pages, p, ex, b, i0, warp, nk, lane);
     };
     const uint64_t policy = evict_first_policy();
     // TMA of one page (K and V of KV head g) into stage k % STAGES; lane 0 only.
@@ -146,19 +142,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     if (p.mode != kModeSparse) {
         setup();
     } else {
-        if (S::kTable > 0 && ex.N <= S::kTable) {
-            // stage the page-table row so that, after the wait, a selected page costs one load
-            for (int j = threadIdx.x; j < ex.N; j += kThreads) table[j] = p.indices[ex.pbeg + j];
-            __syncthreads();
-            ex.table = table;
-        }
         const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
         const int scnt = min(max(p.sel_cnt[b], 0), cap);
         const int si0 = split * p.items_per_split;
         const int si1 = min(si0 + p.items_per_split, scnt);
-        nk_spec = (si1 - si0 > warp) ? (si1 - si0 - warp + kWarps - 1) / kWarps : 0;
+        nk_spec = (si1 - si0 > warp) ? (si1 - si0 - warp + WARPS - 1) / WARPS : 0;
         spec.cur = 0;
-        fetch_pages<true>(p, ex, b, si0, warp, nk_spec, 0, lane, spec.lp_a, spec.ph_a);
+        fetch_pages<true, WARPS>(p, ex, b, si0, warp, nk_spec, 0, lane, spec.lp_a, spec.ph_a);
         spec.lp_b = spec.ph_b = -1;
     }
     {
@@ -196,21 +186,21 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
         // The selection's entries at the speculated positions are loaded together with its count
         // (one round trip); they are the real ones whenever the count is the speculated one.
         const int lp_real = (lane < nk_spec)
-                                ? p.sel_pages[size_t(b) * p.sel_stride + split * p.items_per_split + warp + lane * kWarps]
+                                ? p.sel_pages[size_t(b) * p.sel_stride + split * p.items_per_split + warp + lane * WARPS]
                                 : -1;
         seq_count(p, b, ex);
         i0 = split * p.items_per_split;
         const int i1 = min(i0 + p.items_per_split, ex.count);
-        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;
+        nk = (i1 - i0 > warp) ? (i1 - i0 - warp + WARPS - 1) / WARPS : 0;
         // The speculation holds if the selection's logical pages of this warp's first chunk are the
         // ones guessed (the page table does not change within the step) and were all valid.
         const bool all_same = __all_sync(0xffffffffu, lane >= nk || (lp_real == spec.lp_a && spec.ph_a >= 0)) &&
                               nk == nk_spec;
         if (all_same) {
             pages = spec;
-            fetch_pages(p, ex, b, i0, warp, nk, 32, lane, pages.lp_b, pages.ph_b);
+            fetch_pages<false, WARPS>(p, ex, b, i0, warp, nk, 32, lane, pages.lp_b, pages.ph_b);
         } else {
-            pages_init(pages, p, ex, b, i0, warp, nk, lane);
+            pages_init<WARPS>(pages, p, ex, b, i0, warp, nk, lane);
             // keep an early load only if it is exactly the selection's page; otherwise drain all
             bool same = nk == nk_spec;
             for (int k = 0; k < min(STAGES, nk_spec); ++k) {
@@ -341,7 +331,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     // Pages are taken two at a time: their QK products, one softmax update and their PV
     // products are independent chains the scheduler interleaves.
     for (int k = 0; k < nk; k += 2) {
-        pages_advance(pages, p, ex, b, i0, warp, nk, lane, k);
+        pages_advance<WARPS>(pages, p, ex, b, i0, warp, nk, lane, k);
         const bool two = k + 1 < nk;
         const int sA = k % STAGES, sB = (k + 1) % STAGES;
         if (!mbar_wait(&wbar[sA], parity(k)) || (two && !mbar_wait(&wbar[sB], parity(k + 1)))) {
@@ -445,7 +435,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const DecodeParams
     __syncthreads();
     constexpr int kPart = STAGES * int(S::kPage) / 4;     // floats between two warps' records
     const float* mo0 = reinterpret_cast<const float*>(smem);
-    merge_epilogue<__nv_bfloat16, D, G, kWarps>(p, smem, mo0, mo0 + kMaxGroup * D, recv, b, g, kPart, kPart,
+    merge_epilogue<__nv_bfloat16, D, G, WARPS, WARPS * 32>(p, smem, mo0, mo0 + kMaxGroup * D, recv, b, g, kPart, kPart,
                                                 (p.mode == kModeDelta) ? mo0 + kMaxGroup * D + kMaxGroup * 2 : nullptr);
 }
 

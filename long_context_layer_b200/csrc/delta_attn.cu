@@ -46,7 +46,7 @@ namespace delta {
 
 // ------------------------------------------------------------------ host side
 constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB each for D = 128), 2 CTAs/SM
-constexpr int kMmaStagesDeep = 6;  // when the whole grid fits one CTA per SM: twice the pages in flight
+constexpr int kMmaWideWarps = 8;   // when a cluster per unit fits one CTA per SM: 8-warp CTAs
 
 struct WsLayout {
     size_t err, tickets, part_ml, part_o, page_lse, split_ml, logits, total;
@@ -99,7 +99,7 @@ int ctas_per_sm(int dtype, int D) {
 // whose partials meet in the workspace.
 struct SplitPlan {
     int cluster, clusters;
-    bool deep;   // one CTA per SM: the deeper-pipelined tensor-core variant
+    bool wide;   // one 8-warp CTA per SM (tensor-core kernel), else 4-warp CTAs, two per SM
     int splits() const { return cluster * clusters; }
 };
 
@@ -115,13 +115,15 @@ int split_target_per_sm(int dtype, int D) {
 // About one wave of CTAs, at least 4 pages per CTA (one per warp).  The splits of one (sequence,
 // KV head) form clusters of at most 16 CTAs that merge through distributed shared memory; only
 // when more than 31 splits pay off do several clusters meet in the workspace.
-SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
+// The plan of one variant (wide: 8-warp CTAs, one per SM).
+SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wide) {
     if (items <= 0) return {1, 1, false};
     const int sms = device_sm_count();
-    const int slots = sms * split_target_per_sm(dtype, D);
     const int units = batch * Hkv;
+    const int warps = wide ? kMmaWideWarps : kWarps;
+    const int slots = wide ? sms : sms * split_target_per_sm(dtype, D);
     int s = slots / (units > 0 ? units : 1);
-    const int cap = (items + kWarps - 1) / kWarps;
+    const int cap = (items + warps - 1) / warps;
     if (s > cap) s = cap;
     if (s > kMaxSplits) s = kMaxSplits;
     static int max_splits = -2;
@@ -134,23 +136,39 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
     SplitPlan pl;
     pl.cluster = s < 16 ? s : 16;
     pl.clusters = s / pl.cluster;
-    // The deep variant (6 stages, one CTA per SM) leaves no room on an SM for the next layer's
-    // CTAs, which then cannot start their first loads while this layer drains; the shallow one
-    // (3 stages, two CTAs per SM) can, and measured faster on every workload, so deep is opt-in.
-    static int deep = -1;
-    if (deep < 0) {
-        const char* e = getenv("DELTA_DEEP");   // tuning override for sweeps
-        deep = (e != nullptr && atoi(e) > 0) ? 1 : 0;
-    }
-    pl.deep = deep && dtype == DELTA_BF16 && int64_t(units) * pl.splits() <= sms;
+    pl.wide = wide;
     return pl;
+}
+
+SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
+    // Few (sequence, KV head) units, so that a full cluster per unit fits one CTA per SM, and at
+    // least two pages per warp of such a cluster: 8-warp CTAs, each warp streaming half the pages
+    // of a 4-warp CTA's warp (the per-warp chain of dependent MMAs, exponentials and shuffles,
+    // not the memory system, bounds such layers).  Short page lists (sparse layers) keep 4-warp
+    // CTAs, two per SM, so the next layer's CTAs find room beside them and start their loads.
+    static int wide_env = -1;
+    if (wide_env < 0) {
+        const char* e = getenv("DELTA_WIDE");   // tuning override for sweeps (0: always 4 warps)
+        wide_env = (e != nullptr && atoi(e) == 0) ? 0 : 1;
+    }
+    const bool wide = wide_env && dtype == DELTA_BF16 && int64_t(batch) * Hkv * 16 <= device_sm_count() &&
+                      items >= 16 * kMmaWideWarps * 2;
+    return plan_variant(dtype, D, batch, Hkv, items, wide);
+}
+
+// Most splits any launch on page lists of at most max_pages can get (workspace bound): both
+// variants' split counts grow with the page count.
+int max_splits_for(int dtype, int D, int batch, int Hkv, int max_pages) {
+    const int a = plan_variant(dtype, D, batch, Hkv, max_pages, false).splits();
+    const int b = plan_variant(dtype, D, batch, Hkv, max_pages, true).splits();
+    return a > b ? a : b;
 }
 
 // with_logits: room for per-token logits of every query head (delta-layers scoring with HEAD_MAX)
 WsLayout ws_layout(const delta_desc* d, int batch, int max_pages, bool with_logits = false) {
     WsLayout w{};
-    // room for as many cluster partials as there are splits (fit_plan never exceeds that)
-    const int S = plan_splits(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages).splits();
+    // room for as many cluster partials as there are splits (fit_plan never exceeds a plan's)
+    const int S = max_splits_for(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages);
     const size_t rows = size_t(batch) * d->num_q_heads;
     size_t off = 0;
     w.err = off;        off += align256(64);
@@ -240,13 +258,13 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const delta_desc* d) {
 
 // ---- kernel selection and cluster occupancy
 template <int D, int G>
-const void* mma_ptr(bool deep, size_t* smem) {
-    if (deep) {
-        *smem = MmaSmem<D, kMmaStagesDeep>::kBytes;
-        return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStagesDeep>);
+const void* mma_ptr(bool wide, size_t* smem) {
+    if (wide) {
+        *smem = MmaSmem<D, kMmaStages, kMmaWideWarps>::kBytes;
+        return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStages, kMmaWideWarps>);
     }
     *smem = MmaSmem<D, kMmaStages>::kBytes;
-    return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStages>);
+    return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStages, kWarps>);
 }
 template <int D, int G>
 const void* simt_ptr(size_t* smem) {
@@ -266,14 +284,14 @@ const void* simt_ptr(size_t* smem) {
         case 8: return CALL(8); \
         default: return nullptr; \
     }
-const void* decode_ptr(int dtype, int D, int G, bool deep, size_t* smem) {
+const void* decode_ptr(int dtype, int D, int G, bool wide, size_t* smem) {
     if (dtype == DELTA_BF16) {
         if (D == 128) {
-#define CALL(g) mma_ptr<128, g>(deep, smem)
+#define CALL(g) mma_ptr<128, g>(wide, smem)
             DELTA_G_PTR(G, CALL)
 #undef CALL
         }
-#define CALL(g) mma_ptr<64, g>(deep, smem)
+#define CALL(g) mma_ptr<64, g>(wide, smem)
         DELTA_G_PTR(G, CALL)
 #undef CALL
     }
@@ -304,7 +322,7 @@ bool configure_kernel(const void* func, size_t smem) {
 }
 
 // Clusters of `cluster` CTAs of this kernel that can be resident at once (cached per device).
-int max_active_clusters(const void* func, size_t smem, int cluster) {
+int max_active_clusters(const void* func, size_t smem, int cluster, int threads) {
     constexpr int kSlots = 512;
     struct Entry { const void* fn; int cluster; int n; };
     static Entry cache[64][kSlots];
@@ -316,7 +334,7 @@ int max_active_clusters(const void* func, size_t smem, int cluster) {
     if (!configure_kernel(func, smem)) return 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster, 1, 1);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -362,11 +380,10 @@ SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) 
         cand.cluster = c;
         cand.clusters = s / c < max_clusters ? s / c : max_clusters;
         if (cand.clusters < 1) continue;
-        cand.deep = pl.deep && int64_t(units) * c * cand.clusters <= device_sm_count();
         size_t smem = 0;
-        const void* fn = decode_ptr(dtype, D, G, cand.deep, &smem);
+        const void* fn = decode_ptr(dtype, D, G, cand.wide, &smem);
         if (fn == nullptr) return pl;
-        const int maxc = max_active_clusters(fn, smem, c);
+        const int maxc = max_active_clusters(fn, smem, c, cand.wide ? kMmaWideWarps * 32 : kThreads);
         if (int64_t(units) * cand.clusters > maxc) {
             cand.clusters = maxc / units;
             if (cand.clusters < 1) continue;
@@ -380,7 +397,7 @@ SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) 
     if (best_ctas < 0) {   // more units than resident clusters even at size 1: several waves
         best.cluster = 1;
         best.clusters = 1;
-        best.deep = false;
+        best.wide = false;
     }
     return best;
 }
@@ -405,12 +422,12 @@ delta_status launch_pdl(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t
 
 // Launch a decode kernel as clusters of `cluster` CTAs along the split dimension.
 template <typename K, typename... Args>
-delta_status launch_clustered(K kern, size_t smem, const DecodeParams& prm, int cluster, int batch, int Hkv,
-                              cudaStream_t st, Args... args) {
+delta_status launch_clustered(K kern, size_t smem, int threads, const DecodeParams& prm, int cluster, int batch,
+                              int Hkv, cudaStream_t st, Args... args) {
     if (!configure_kernel(reinterpret_cast<const void*>(kern), smem)) return DELTA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(prm.num_splits, Hkv, batch);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -429,18 +446,19 @@ delta_status launch_clustered(K kern, size_t smem, const DecodeParams& prm, int 
 template <typename T, int D, int G>
 delta_status launch_simt_g(const DecodeParams& prm, int cluster, int batch, int Hkv, cudaStream_t st) {
     constexpr int STAGES = simt_stages(int(sizeof(T)), D);
-    return launch_clustered(decode_kernel<T, D, G, STAGES>, DecodeSmem<T, D, STAGES>::kBytes, prm, cluster, batch, Hkv,
-                            st);
+    return launch_clustered(decode_kernel<T, D, G, STAGES>, DecodeSmem<T, D, STAGES>::kBytes, kThreads, prm, cluster,
+                            batch, Hkv, st);
 }
 
 template <int D, int G>
 delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const CUtensorMap& mv, int cluster,
-                          bool deep, int batch, int Hkv, cudaStream_t st) {
-    if (deep)
-        return launch_clustered(decode_mma_kernel<D, G, kMmaStagesDeep>, MmaSmem<D, kMmaStagesDeep>::kBytes, prm,
-                                cluster, batch, Hkv, st, mk, mv);
-    return launch_clustered(decode_mma_kernel<D, G, kMmaStages>, MmaSmem<D, kMmaStages>::kBytes, prm, cluster, batch,
-                            Hkv, st, mk, mv);
+                          bool wide, int batch, int Hkv, cudaStream_t st) {
+    if (wide)
+        return launch_clustered(decode_mma_kernel<D, G, kMmaStages, kMmaWideWarps>,
+                                MmaSmem<D, kMmaStages, kMmaWideWarps>::kBytes, kMmaWideWarps * 32, prm, cluster, batch,
+                                Hkv, st, mk, mv);
+    return launch_clustered(decode_mma_kernel<D, G, kMmaStages, kWarps>, MmaSmem<D, kMmaStages>::kBytes, kThreads, prm,
+                            cluster, batch, Hkv, st, mk, mv);
 }
 
 #define DELTA_G_SWITCH(G, CALL) \
@@ -456,18 +474,18 @@ delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const 
         default: return DELTA_ERR_UNSUPPORTED; \
     }
 
-delta_status launch_decode(const delta_desc* d, const DecodeParams& prm, int cluster, bool deep, int batch,
+delta_status launch_decode(const delta_desc* d, const DecodeParams& prm, int cluster, bool wide, int batch,
                            cudaStream_t st) {
     const int Hkv = d->num_kv_heads, G = d->num_q_heads / Hkv;
     if (d->dtype == DELTA_BF16) {
         CUtensorMap mk, mv;
         if (!make_pool_map(&mk, prm.k_pool, d) || !make_pool_map(&mv, prm.v_pool, d)) return DELTA_ERR_CUDA;
         if (d->head_dim == 128) {
-#define CALL(g) launch_mma_g<128, g>(prm, mk, mv, cluster, deep, batch, Hkv, st)
+#define CALL(g) launch_mma_g<128, g>(prm, mk, mv, cluster, wide, batch, Hkv, st)
             DELTA_G_SWITCH(G, CALL)
 #undef CALL
         } else {
-#define CALL(g) launch_mma_g<64, g>(prm, mk, mv, cluster, deep, batch, Hkv, st)
+#define CALL(g) launch_mma_g<64, g>(prm, mk, mv, cluster, wide, batch, Hkv, st)
             DELTA_G_SWITCH(G, CALL)
 #undef CALL
         }
@@ -552,7 +570,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.tickets = reinterpret_cast<int*>(base + L.tickets);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    s = launch_decode(d, prm, plan.cluster, plan.deep, pt->batch, st);
+    s = launch_decode(d, prm, plan.cluster, plan.wide, pt->batch, st);
     if (s != DELTA_OK || mode != kModeDelta) return s;
 
     SelectParams sp2{};
