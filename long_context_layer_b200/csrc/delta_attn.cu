@@ -132,6 +132,12 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wid
         max_splits = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
     }
     if (max_splits > 0 && s > max_splits) s = max_splits;
+    static int max_wide = -2;
+    if (max_wide == -2) {
+        const char* e = getenv("DELTA_MAX_WIDE_SPLITS");   // tuning override for sweeps
+        max_wide = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
+    }
+    if (wide && max_wide > 0 && s > max_wide) s = max_wide;
     if (s < 1) s = 1;
     SplitPlan pl;
     pl.cluster = s < 16 ? s : 16;
