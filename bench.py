@@ -62,10 +62,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the full-layer decode from the committed ncu summary of this
-    workload, or None when the kernels changed since that capture."""
-    path = os.path.join(ROOT, "profiles", f"decode_full_layer_{workload}.md")
+def profiled_traffic(workload: str, kind: str = "full_layer"):
+    """DRAM bytes per launch of the decode kernel in a full or sparse layer, from the committed ncu
+    summary of this workload, or None when the kernels changed since that capture."""
+    path = os.path.join(ROOT, "profiles", f"decode_{kind}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
@@ -470,6 +470,26 @@ def run_ours(args):
         NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[ls], dc.k_pools[ls],
                         dc.v_pools[ls], dc.out[ls], d0.workspace, d0.ws_bytes, st)
 
+    # -- the sparse-layer decode (24 of the 28 launches of a step): L launches of it in one graph,
+    #    all on the delta-layer's selection, timed like the steps; per-launch average
+    lay = list(range(cfg.num_layers))
+    sg = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for l in lay:   # warm outside capture (per-device kernel attributes)
+            NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[l], dc.k_pools[l],
+                            dc.v_pools[l], dc.out[l], d0.workspace, d0.ws_bytes, side.cuda_stream)
+    stream.wait_stream(side)
+    with torch.cuda.graph(sg):
+        cs = torch.cuda.current_stream(device).cuda_stream
+        for l in lay:
+            NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[l], dc.k_pools[l],
+                            dc.v_pools[l], dc.out[l], d0.workspace, d0.ws_bytes, cs)
+    t_sparse = timed(sg.replay, max(args.steps // 2, 10), 3)
+    us_sparse_launch = max_over_ranks(dist, statistics.mean(t_sparse), device) / len(lay)
+    del sg
+
     n_b = max(args.steps // 2, 10)
     breakdown = {name: round(max_over_ranks(dist, statistics.mean(timed(fn, n_b, 3)), device), 3)
                  for name, fn in (("kv_append", append_call), ("full_attn", full_call),
@@ -486,6 +506,11 @@ def run_ours(args):
     us_launch = us_full / cfg.num_layers
     achieved = alg_bytes / (us_launch * 1e-6) / 1e9
     achieved_single = alg_bytes / (us_kernel * 1e-6) / 1e9
+    # sparse layers: the tokens of the selected pages of every sequence
+    _, _, _, sparse_tok = attended_tokens(cfg, case)
+    alg_sparse = sparse_tok * 2 * cfg.num_kv_heads * cfg.head_dim * e + qo_bytes
+    achieved_sparse = alg_sparse / (us_sparse_launch * 1e-6) / 1e9
+    n_sparse = kinds.count("sparse")
 
     # -- end to end through the public API: pinned host inputs in, outputs out, every step
     q_h = dc.q.cpu().pin_memory()
@@ -532,14 +557,24 @@ def run_ours(args):
             "full_stack_us": round(us_full, 3),
             "speedup_vs_full_stack": round(us_full / us_delta, 3),
             "attended_token_reduction": round(tok_full / tok_delta, 3),
-            "roofline": {"kernel": "decode_mma_kernel, full layer (split-KV, cluster merge)", "bound": "hbm",
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                         "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_launch, 3),
-                         "timing": "full-attention stack graph (L launches + 1 append) / L, CUDA events, L2 flushed",
-                         "single_call_us": round(us_kernel, 3),
-                         "single_call_frac": round(achieved_single / peak, 4),
-                         "traffic": profiled_traffic(cfg.name)},
+            # the kernel that dominates the step: the decode kernel of the sparse layers
+            "roofline": {"kernel": "decode_mma_kernel, sparse layer (selected pages, split-KV, cluster merge)",
+                         "bound": "hbm", "achieved": round(achieved_sparse, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved_sparse / peak, 4), "peak_source": peak_kind,
+                         "alg_bytes_per_launch": alg_sparse, "us_per_launch": round(us_sparse_launch, 3),
+                         "launches_per_step": n_sparse,
+                         "share_of_step": round(n_sparse * us_sparse_launch / us_delta, 3),
+                         "timing": "graph of L sparse launches on the delta-layer's selection / L, CUDA events, L2 flushed",
+                         "traffic": profiled_traffic(cfg.name, "sparse_layer")},
+            "roofline_full_layer": {"kernel": "decode_mma_kernel, full layer (split-KV, cluster merge)", "bound": "hbm",
+                                    "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                                    "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                                    "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_launch, 3),
+                                    "launches_per_step": len(kinds) - n_sparse,
+                                    "timing": "full-attention stack graph (L launches + 1 append) / L, CUDA events, L2 flushed",
+                                    "single_call_us": round(us_kernel, 3),
+                                    "single_call_frac": round(achieved_single / peak, 4),
+                                    "traffic": profiled_traffic(cfg.name, "full_layer")},
             "breakdown_us_per_call": breakdown,
             "e2e": {"value": round(us_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
