@@ -94,9 +94,9 @@ int ctas_per_sm(int dtype, int D) {
     return c < 1 ? 1 : (c > 8 ? 8 : c);
 }
 
-// Split plan: about one full wave of CTAs over the GPU, at least 4 pages per CTA (one per
-// warp).  Up to 16 splits form one thread-block cluster; more are grouped into clusters of 8
-// whose partials meet in the workspace.
+// Split plan: about one full wave of CTAs over the GPU, at least one page per warp.  Up to 16
+// splits form one thread-block cluster; more are grouped into clusters whose partials meet in the
+// workspace.
 struct SplitPlan {
     int cluster, clusters;
     bool wide;   // one 8-warp CTA per SM (tensor-core kernel), else 4-warp CTAs, two per SM
@@ -112,9 +112,9 @@ int split_target_per_sm(int dtype, int D) {
     return override_ > 0 ? override_ : ctas_per_sm(dtype, D);
 }
 
-// About one wave of CTAs, at least 4 pages per CTA (one per warp).  The splits of one (sequence,
-// KV head) form clusters of at most 16 CTAs that merge through distributed shared memory; only
-// when more than 31 splits pay off do several clusters meet in the workspace.
+// About one wave of CTAs, at least one page per warp.  The splits of one (sequence, KV head) form
+// clusters of at most 16 CTAs that merge through distributed shared memory; only long page lists
+// (fit_plan) make several clusters meet in the workspace.
 // The plan of one variant (wide: 8-warp CTAs, one per SM).
 SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wide) {
     if (items <= 0) return {1, 1, false};
@@ -138,6 +138,12 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wid
         max_wide = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
     }
     if (wide && max_wide > 0 && s > max_wide) s = max_wide;
+    static int max_narrow = -2;
+    if (max_narrow == -2) {
+        const char* e = getenv("DELTA_MAX_NARROW_SPLITS");   // tuning override for sweeps
+        max_narrow = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
+    }
+    if (!wide && max_narrow > 0 && s > max_narrow) s = max_narrow;
     if (s < 1) s = 1;
     SplitPlan pl;
     pl.cluster = s < 16 ? s : 16;
