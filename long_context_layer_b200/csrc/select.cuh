@@ -238,12 +238,9 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     uint32_t T = 0, need_eq = 0;
     if (!take_all && k > 0 && C == 1) {
         // one CTA: bucket b(key) = (key - kmin) >> sh in [0, 255] (monotone in the key)
-        uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll 8
-        for (int w = 0; w < kSelectThreads / 32; ++w) {
-            kmin = min(kmin, s_kmin[w]);
-            kmax = max(kmax, s_kmax[w]);
-        }
+        // every warp combines the 32 per-warp values itself: one load per lane, not 64 per thread
+        const uint32_t kmin = __reduce_min_sync(0xffffffffu, s_kmin[lane]);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, s_kmax[lane]);
         const uint32_t span = kmax - kmin;   // ncand > k >= 1 candidates: kmin <= kmax
         const int sh = max(0, 24 - __clz(span));
         // warp-aggregated: most keys crowd into a few buckets, so lanes of one bucket add once
