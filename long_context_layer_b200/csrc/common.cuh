@@ -327,10 +327,10 @@ __device__ __forceinline__ void merge_prologue(float* recv) {
     cluster_wait();
 }
 
-// Part rr's records: outputs mo[rr * ostride + h * D + d], states ml[rr * mstride + 2 * h] (max,
+// Part rr's records: outputs mo[rr * ostride + h * OROW + d], states ml[rr * mstride + 2 * h] (max,
 // sum) of base-2 logits; dml (delta-layers, same strides as ml) holds the states over the exact
 // fp32 page terms when those differ from ml.
-template <typename T, int D, int G, int NPART, int NTHR = kThreads>
+template <typename T, int D, int G, int NPART, int NTHR = kThreads, int OROW = D>
 __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned char* smem, const float* mo,
                                                const float* mml, float* recv, int b, int g, int ostride,
                                                int mstride, const float* dml = nullptr) {
@@ -393,7 +393,7 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
 #pragma unroll
         for (int rr = 0; rr < NPART; ++rr) {
             const float w = exp2_approx(mml[rr * mstride + 2 * h] - mu);
-            const float4 v = *reinterpret_cast<const float4*>(&mo[rr * ostride + h * D + d]);
+            const float4 v = *reinterpret_cast<const float4*>(&mo[rr * ostride + h * OROW + d]);
             acc.x = fmaf(w, v.x, acc.x);
             acc.y = fmaf(w, v.y, acc.y);
             acc.z = fmaf(w, v.z, acc.z);

@@ -65,7 +65,7 @@ struct MmaSmem {
     static constexpr uint32_t kPage = 2 * kBoxes * kBox;      // K and V of one page, one KV head
     static constexpr size_t kStages = size_t(WARPS) * STAGES * kPage;
     // each warp's merge record ([8][D] outputs, two [8][2] states) reuses its own stages
-    static_assert(size_t(STAGES) * kPage >= (size_t(kMaxGroup) * D + 4 * kMaxGroup) * sizeof(float), "merge record");
+    static_assert(size_t(STAGES) * kPage >= (size_t(kMaxGroup) * (D + 4) + 4 * kMaxGroup) * sizeof(float), "merge record");
     static constexpr size_t kMain = kStages;
     static constexpr size_t kBars = size_t(WARPS) * STAGES * sizeof(uint64_t);
     static constexpr size_t kRecv = size_t(recv_floats<D>()) * sizeof(float);
@@ -409,16 +409,18 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
     // ---- this warp's state into its own stage area (all of its copies have landed and no other
     // warp touches that area), one barrier, then the merge of the 4 warps and of the splits
     __syncwarp();
-    float* po = reinterpret_cast<float*>(wst);           // [8][D] outputs
-    float* pml = po + kMaxGroup * D;                      // [8][2] (max, sum)
+    // rows padded by 4 floats: the four lanes of a column group (t4) store to different banks
+    constexpr int kRow = D + 4;
+    float* po = reinterpret_cast<float*>(wst);           // [8][D + 4] outputs
+    float* pml = po + kMaxGroup * kRow;                   // [8][2] (max, sum)
     float* pdl = pml + kMaxGroup * 2;                     // [8][2] delta-layers: over the fp32 page terms
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) {
         const int d = mt * 16 + g4;
-        po[(2 * t4) * D + d] = acc[mt][0];
-        po[(2 * t4 + 1) * D + d] = acc[mt][1];
-        po[(2 * t4) * D + d + 8] = acc[mt][2];
-        po[(2 * t4 + 1) * D + d + 8] = acc[mt][3];
+        po[(2 * t4) * kRow + d] = acc[mt][0];
+        po[(2 * t4 + 1) * kRow + d] = acc[mt][1];
+        po[(2 * t4) * kRow + d + 8] = acc[mt][2];
+        po[(2 * t4 + 1) * kRow + d + 8] = acc[mt][3];
     }
     if (g4 == 0) {
         pml[(2 * t4) * 2 + 0] = m_run[0];
@@ -435,8 +437,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
     __syncthreads();
     constexpr int kPart = STAGES * int(S::kPage) / 4;     // floats between two warps' records
     const float* mo0 = reinterpret_cast<const float*>(smem);
-    merge_epilogue<__nv_bfloat16, D, G, WARPS, WARPS * 32>(p, smem, mo0, mo0 + kMaxGroup * D, recv, b, g, kPart, kPart,
-                                                (p.mode == kModeDelta) ? mo0 + kMaxGroup * D + kMaxGroup * 2 : nullptr);
+    merge_epilogue<__nv_bfloat16, D, G, WARPS, WARPS * 32, kRow>(
+        p, smem, mo0, mo0 + kMaxGroup * kRow, recv, b, g, kPart, kPart,
+        (p.mode == kModeDelta) ? mo0 + kMaxGroup * kRow + kMaxGroup * 2 : nullptr);
 }
 
 }  // namespace delta
