@@ -124,27 +124,27 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     const int sub = tid & 1;
 
     // 1. per-head normaliser from the splits' states, a warp per head: the maximum first, then the
-    //    rescaled sum, so the exponentials are independent (no serial online update)
+    //    rescaled sum, so the exponentials are independent (no serial online update); four states
+    //    per lane and round, no exponential for an empty slot
     for (int h = warp; h < Hq; h += kSelectThreads / 32) {
         const float2* ps = p.split_ml + (size_t(b) * Hq + h) * p.num_splits;
         float M = -INFINITY, Z = 0.f;
-        for (int base = 0; base < p.num_splits; base += 32 * 16) {   // one round up to 512 splits
-            float2 v[16];
+        for (int base = 0; base < p.num_splits; base += 32 * 4) {
+            float2 v[4];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 const int s = base + lane + 32 * u;
                 v[u] = (s < p.num_splits) ? ps[s] : make_float2(-INFINITY, 0.f);
             }
-            float Mr = v[0].x;
-#pragma unroll
-            for (int u = 1; u < 16; ++u) Mr = fmaxf(Mr, v[u].x);
+            float Mr = fmaxf(fmaxf(v[0].x, v[1].x), fmaxf(v[2].x, v[3].x));
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
             const float Mn = fmaxf(M, Mr);
             const float mu = (Mn == -INFINITY) ? 0.f : Mn;
             float z = 0.f;
 #pragma unroll
-            for (int u = 0; u < 16; ++u) z = fmaf(v[u].y, exp2_approx(v[u].x - mu), z);
+            for (int u = 0; u < 4; ++u)
+                if (v[u].y > 0.f) z = fmaf(v[u].y, exp2_approx(v[u].x - mu), z);
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
             Z = Z * exp2_approx(M - mu) + z;
@@ -243,13 +243,8 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
         const uint32_t kmax = __reduce_max_sync(0xffffffffu, s_kmax[lane]);
         const uint32_t span = kmax - kmin;   // ncand > k >= 1 candidates: kmin <= kmax
         const int sh = max(0, 24 - __clz(span));
-        // warp-aggregated: most keys crowd into a few buckets, so lanes of one bucket add once
-        for (int base = j0; base < j1; base += kSelectThreads) {   // uniform trip count
-            const int j = base + tid;
-            const uint32_t bk = (j < j1 && !forced(j)) ? (keys[j - j0] - kmin) >> sh : 0xffffffffu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, bk);
-            if (bk != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[0][bk], uint32_t(__popc(peers)));
-        }
+        for (int j = j0 + tid; j < j1; j += kSelectThreads)
+            if (!forced(j)) atomicAdd(&hist[0][(keys[j - j0] - kmin) >> sh], 1u);
         __syncthreads();
         if (tid < 32) {   // the bucket holding the k-th largest, and the keys in higher buckets
             uint32_t c[8], sum = 0;
