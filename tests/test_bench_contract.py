@@ -1,0 +1,47 @@
+"""Host-side checks of bench.py: the reference arm's JSON line and the attended-token accounting
+that the roofline's algorithmic bytes are built from (no GPU needed)."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+from oracle import delta_oracle as O
+from synth import configs as C
+from synth.case import Case
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "1",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["higher_is_better"] is False and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == C.TINY.name
+
+
+def test_attended_tokens_match_the_oracle_selection():
+    # the sparse-layer token count the roofline uses equals the tokens of the oracle's selection
+    import bench
+    for cfg in (C.TINY, C.QWEN7B_8K.with_(context=8192 - 5)):
+        case = Case(cfg)
+        delta_tok, full_tok_stack, full_tok, sparse_tok = bench.attended_tokens(cfg, case)
+        n = int(case.n[0])
+        S = np.zeros(-(-n // 16))   # scores do not change the count: ties keep k candidates
+        sel = O.select_pages(S, n, 16, cfg.budget_pages, cfg.sink_tokens, cfg.recency_tokens)
+        assert sparse_tok == len(O.page_tokens(sel, n, 16))
+        assert full_tok == n
+        kinds = cfg.layer_kinds()
+        assert full_tok_stack == len(kinds) * n
+        assert delta_tok == kinds.count("sparse") * sparse_tok + (len(kinds) - kinds.count("sparse")) * n
