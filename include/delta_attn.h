@@ -4,9 +4,9 @@
  * DELTA ("DELTA: Dynamic Layer-Aware Token Attention for Efficient Long-Context
  * Reasoning", ai.info summary, section "Methodology in Plain English") splits a
  * model's layers into initial full-attention layers, a few delta-layers that run
- * full attention and score the KV pages, and sparse layers that attend only to the
- * pages the latest delta-layer selected.  The KV cache is kept in full and paged
- * with 16-token pages (same section: "a fixed page size of 16").  This header
+ * full attention and rank the KV pages, and sparse layers that read only the pages
+ * chosen by the most recent delta-layer.  The whole KV cache stays in memory, paged
+ * 16 tokens to a page (same section).  This header
  * exposes one call per step of that decode path:
  *
  *   delta_kv_append    write the current token's k, v into the paged cache
@@ -72,9 +72,10 @@ typedef enum { DELTA_F32 = 0, DELTA_BF16 = 1 } delta_dtype;
 /* How per-token attention is aggregated over query heads for the page score. */
 typedef enum {
     DELTA_HEAD_SUM = 0,  /* S_j = sum over query heads h and tokens t of page j of p[h][t] */
-    DELTA_HEAD_MAX = 1   /* S_j = sum over tokens t of page j of max_h p[h][t] ("for each token they take
-                            the maximum attention weight across heads", ai.info summary, "Methodology in
-                            Plain English"); needs delta_workspace_size_reduce(..., DELTA_HEAD_MAX) */
+    DELTA_HEAD_MAX = 1   /* S_j = sum over tokens t of page j of max_h p[h][t] (the page's own rule: a
+                            token's weight is its largest attention weight over the heads; ai.info summary,
+                            "Methodology in Plain English"); needs delta_workspace_size_reduce(...,
+                            DELTA_HEAD_MAX) */
 } delta_head_reduce;
 
 /* Shape of one attention layer.  Supported: head_dim 64 or 128, page_size 16,
@@ -130,8 +131,8 @@ int32_t delta_sel_capacity(const delta_select_params* sp, int32_t page_size);
 /* Write token kv_len[b]-1 of every sequence: k_new[b][g] and v_new[b][g] go to slot
  * (kv_len[b]-1) % page_size of logical page (kv_len[b]-1) / page_size.  The page
  * must already be in the page table.  Sequences with kv_len 0 are skipped.  The
- * rest of the cache is never modified ("DELTA never removes tokens from the KV
- * cache", ai.info summary, "Methodology in Plain English"). */
+ * rest of the cache is never modified (DELTA evicts nothing from the cache; ai.info
+ * summary, "Methodology in Plain English"). */
 delta_status delta_kv_append(const delta_desc* desc, const delta_page_table* pt,
                              const void* k_new, const void* v_new,
                              void* k_pool, void* v_pool, void* stream);
@@ -145,8 +146,8 @@ delta_status delta_kv_append_layers(const delta_desc* desc, const delta_page_tab
                                     void* const* k_pools, void* const* v_pools, void* stream);
 
 /* Full decode attention: o[b][h] = sum_t softmax_t(sm_scale * q[b][h].k_t) v_t over the
- * kv_len[b] cached tokens of KV head h/G (initial layers "run ordinary full attention",
- * ai.info summary, "Methodology in Plain English").  kv_len 0 gives o = 0. */
+ * kv_len[b] cached tokens of KV head h/G (the initial layers of the stack; ai.info summary,
+ * "Methodology in Plain English").  kv_len 0 gives o = 0. */
 delta_status delta_full_attn(const delta_desc* desc, const delta_page_table* pt,
                              const void* q, const void* k_pool, const void* v_pool, void* o,
                              void* workspace, size_t ws_bytes, void* stream);
@@ -189,9 +190,9 @@ delta_status delta_select_attn(const delta_desc* desc, const delta_page_table* p
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* Sparse layer: attention restricted to the tokens (< kv_len[b]) of the logical pages
- * sel_pages[b][0..sel_cnt[b]), softmax renormalised over them ("Every remaining layer
- * then runs sparse attention, attending only to the tokens in those selected pages",
- * ai.info summary, "Methodology in Plain English").  Pages are mapped through the
+ * sel_pages[b][0..sel_cnt[b]), softmax renormalised over them (the layers after a
+ * delta-layer read only the pages it selected; ai.info summary, "Methodology in Plain
+ * English").  Pages are mapped through the
  * page table, so one selection serves every layer's pools. */
 delta_status delta_sparse_attn(const delta_desc* desc, const delta_page_table* pt,
                                const int32_t* sel_cnt, const int32_t* sel_pages, int32_t sel_stride,
@@ -200,10 +201,11 @@ delta_status delta_sparse_attn(const delta_desc* desc, const delta_page_table* p
 
 /* Delta-layer calibration metric: shift_out[b] = 1 - cos(scores_a[b], scores_b[b]) over the
  * pages j < ceil(kv_len[b]/page_size) of two layers' page scores (the page_scores outputs of
- * delta_select_attn, [batch][max_pages_per_seq] fp32).  The calibration picks delta-layers
- * from the average shift between consecutive layers, "1 - cosine similarity averaged over
- * decoding steps and samples" (ai.info summary, "Methodology in Plain English"); a layer's
- * attention map is read as its page-score vector.  A zero vector gives a shift of 1. */
+ * delta_select_attn, [batch][max_pages_per_seq] fp32).  The calibration places delta-layers
+ * where consecutive layers' attention differs most, the difference being one minus their
+ * cosine similarity, averaged by the caller over steps and inputs (ai.info summary,
+ * "Methodology in Plain English"); a layer's attention map is read as its page-score vector.
+ * A zero vector gives a shift of 1. */
 delta_status delta_layer_shift(const delta_page_table* pt, const float* scores_a, const float* scores_b,
                                float* shift_out, void* stream);
 

@@ -115,7 +115,7 @@ class DeltaStack:
 
         Every layer from 1 on runs as a delta-layer (full attention plus page scores) on the
         current cache; layers 0 and 1 get shift 0.  DELTA's calibration (ai.info summary,
-        "Methodology in Plain English") averages such shifts over decoding steps and samples
+        "Methodology in Plain English") averages such shifts over several steps and inputs
         and places the delta-layers where they are large.
         """
         st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream

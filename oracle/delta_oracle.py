@@ -13,7 +13,7 @@ a step open:
   token's query against every cached token (scale 1/sqrt(D), no mask beyond
   the context length, the current token included);
 * grouped-query attention: query head h reads KV head h // G, G = Hq / Hkv;
-* a delta-layer's own output is full attention ("also run full attention");
+* a delta-layer's own output is full attention (it attends to every token while scoring);
 * the page score is the softmax probability summed over all query heads of
   the sequence and over the page's tokens (HEAD_SUM).  The page's own wording,
   the maximum weight across heads per token summed over the page, is kept as

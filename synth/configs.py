@@ -9,8 +9,8 @@ Qwen-7B / Llama-8B / Qwen-14B-shaped stacks follow the calibrated lists under
 "Main Findings" (the last bullet) of the same page where the workload names them.
 
 Token/page arithmetic follows the same page ("Main Findings", fifth bullet):
-a budget of K pages of P=16 tokens is K*16 tokens, e.g. 64 pages = 1k tokens,
-and a recency window of L=8 pages is 128 tokens.
+a budget of K pages of P=16 tokens is K*16 tokens (64 pages are 1k tokens), and
+the recency window of 8 pages covers 128 tokens.
 """
 from __future__ import annotations
 
