@@ -13,7 +13,8 @@
  *                      (delta_kv_append_layers: every layer of a step in one launch)
  *   delta_full_attn    full decode attention (initial layers)
  *   delta_select_attn  full decode attention + per-page scores + page selection (delta-layers)
- *   delta_sparse_attn  decode attention over the selected pages only (sparse layers)
+ *   delta_sparse_attn  decode attention over the selected pages only (sparse layers);
+ *                      delta_sparse_attn_settled when the selection was final one kernel earlier
  *
  * Conventions shared by every call
  * --------------------------------
@@ -198,6 +199,19 @@ delta_status delta_sparse_attn(const delta_desc* desc, const delta_page_table* p
                                const int32_t* sel_cnt, const int32_t* sel_pages, int32_t sel_stride,
                                const void* q, const void* k_pool, const void* v_pool, void* o,
                                void* workspace, size_t ws_bytes, void* stream);
+
+/* delta_sparse_attn for a settled selection: the caller states that sel_cnt, sel_pages, the
+ * pools and the page table were final before the kernel that precedes this call in `stream`
+ * began (in a decode step: every sparse layer but the first after the delta-layer that wrote
+ * the selection, since that first one directly follows the selection kernel).  The kernel
+ * then reads the selection and loads its pages, the appended token's page included, before
+ * waiting on the preceding kernel, instead of loading the selection again after the wait to
+ * check a guess.  Same arguments, output, errors and device flags as delta_sparse_attn; a
+ * call that breaks the statement may read a stale selection or page. */
+delta_status delta_sparse_attn_settled(const delta_desc* desc, const delta_page_table* pt,
+                                       const int32_t* sel_cnt, const int32_t* sel_pages, int32_t sel_stride,
+                                       const void* q, const void* k_pool, const void* v_pool, void* o,
+                                       void* workspace, size_t ws_bytes, void* stream);
 
 /* Delta-layer calibration metric: shift_out[b] = 1 - cos(scores_a[b], scores_b[b]) over the
  * pages j < ceil(kv_len[b]/page_size) of two layers' page scores (the page_scores outputs of

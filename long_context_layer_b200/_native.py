@@ -27,6 +27,7 @@ EXPORTED = [
     "delta_workspace_size", "delta_workspace_size_reduce", "delta_workspace_init", "delta_sel_capacity", "delta_kv_append",
     "delta_kv_append_layers",
     "delta_full_attn", "delta_full_attn_noalloc", "delta_select_attn", "delta_sparse_attn",
+    "delta_sparse_attn_settled",
     "delta_layer_shift", "delta_read_device_error",
     "delta_status_string",
 ]
@@ -74,6 +75,8 @@ lib.delta_select_attn.argtypes = [_D, _PT, _SP, _vp, _vp, _vp, _vp, _vp, _vp, _i
 lib.delta_select_attn.restype = _i32
 lib.delta_sparse_attn.argtypes = [_D, _PT, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.delta_sparse_attn.restype = _i32
+lib.delta_sparse_attn_settled.argtypes = [_D, _PT, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.delta_sparse_attn_settled.restype = _i32
 lib.delta_layer_shift.argtypes = [_PT, _vp, _vp, _vp, _vp]
 lib.delta_layer_shift.restype = _i32
 lib.delta_read_device_error.argtypes = [_vp, ctypes.POINTER(_i32), _vp]
@@ -168,6 +171,13 @@ def sparse_attn(desc, pt, sel_cnt, sel_pages, sel_stride: int, q, k_pool, v_pool
     s = lib.delta_sparse_attn(ctypes.byref(desc), ctypes.byref(pt), ptr(sel_cnt), ptr(sel_pages), sel_stride,
                               ptr(q), ptr(k_pool), ptr(v_pool), ptr(o), ptr(workspace), ws_bytes, stream)
     return _check(s, "delta_sparse_attn") if check else s
+
+
+def sparse_attn_settled(desc, pt, sel_cnt, sel_pages, sel_stride: int, q, k_pool, v_pool, o, workspace,
+                        ws_bytes: int, stream: int = 0, check: bool = True) -> int:
+    s = lib.delta_sparse_attn_settled(ctypes.byref(desc), ctypes.byref(pt), ptr(sel_cnt), ptr(sel_pages), sel_stride,
+                                      ptr(q), ptr(k_pool), ptr(v_pool), ptr(o), ptr(workspace), ws_bytes, stream)
+    return _check(s, "delta_sparse_attn_settled") if check else s
 
 
 def layer_shift(pt, scores_a, scores_b, shift_out, stream: int = 0, check: bool = True) -> int:

@@ -192,6 +192,9 @@ struct DecodeParams {
     float2* split_ml; // [B][Hq][S] (max, sum) of each split CTA's own pages (delta-layers)
     void* o;          // [B][Hq][D] output
     int32_t num_clusters;   // clusters along the split dimension (num_splits = cluster size * this)
+    // sparse layers: the selection, pools and page table were final before the previous kernel
+    // of the stream began, so they are read (and the pages loaded) before waiting on it
+    int32_t settled;
     float* logits;          // [B][Hq][max_pages*16] base-2 logits (delta-layers in HEAD_MAX mode), else null
     int* tickets;     // [B][Hkv] arrival counters of the split CTAs, zero between launches
     int* err;
@@ -233,7 +236,8 @@ __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int
     ph = -1;
     if (k >= nk) return;
     const int i = i0 + warp + k * W;
-    lp = (p.mode == kModeSparse) ? p.sel_pages[size_t(b) * p.sel_stride + i] : i;
+    // the selection is read from L2 (another kernel of the step wrote it; no stale L1 line)
+    lp = (p.mode == kModeSparse) ? __ldcg(p.sel_pages + size_t(b) * p.sel_stride + i) : i;
     if (lp < 0 || lp >= ex.N) {
         if (!QUIET) atomicOr(p.err, kErrSel);
         lp = -1;
@@ -298,7 +302,7 @@ __device__ __forceinline__ SeqExtent seq_extent(const P& p, int b) {
 template <typename P>
 __device__ __forceinline__ void seq_count(const P& p, int b, SeqExtent& ex) {
     if (p.mode != kModeSparse) return;
-    const int scnt = p.sel_cnt[b];
+    const int scnt = __ldcg(p.sel_cnt + b);
     const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
     ex.count = scnt;
     if (scnt < 0 || scnt > cap) {

@@ -102,8 +102,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
     __syncwarp();
     merge_prologue(recv);
     // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
-    // so full and delta layers resolve their pages before waiting for the previous kernel; the
-    // sparse layers' page list is the output of the delta-layer and is read after the wait.
+    // so full and delta layers resolve their pages before waiting for the previous kernel; a
+    // sparse layer's page list is the output of the delta-layer: read before the wait when the
+    // caller states it settled, else speculated on before the wait and checked after it.
     SeqExtent ex = seq_extent(p, b);
     int i0 = 0, nk = 0;
     WarpPages pages;
@@ -139,11 +140,11 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
     uint32_t spec_used = 0;   // bit s: stage s spent its first phase on a discarded speculative load
     WarpPages spec;
     int nk_spec = 0;
-    if (p.mode != kModeSparse) {
-        setup();
+    if (p.mode != kModeSparse || p.settled) {
+        setup();   // a settled selection is final: read (and checked) now
     } else {
         const int cap = min(p.sel_stride, p.items_per_split * p.num_splits);
-        const int scnt = min(max(p.sel_cnt[b], 0), cap);
+        const int scnt = min(max(__ldcg(p.sel_cnt + b), 0), cap);
         const int si0 = split * p.items_per_split;
         const int si1 = min(si0 + p.items_per_split, scnt);
         nk_spec = (si1 - si0 > warp) ? (si1 - si0 - warp + WARPS - 1) / WARPS : 0;
@@ -152,12 +153,14 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
         spec.lp_b = spec.ph_b = -1;
     }
     {
-        const WarpPages& pre = (p.mode == kModeSparse) ? spec : pages;
-        const int npre = min(STAGES, (p.mode == kModeSparse) ? nk_spec : nk);
+        const bool speculative = p.mode == kModeSparse && !p.settled;
+        const WarpPages& pre = speculative ? spec : pages;
+        const int npre = min(STAGES, speculative ? nk_spec : nk);
         for (int k = 0; k < npre; ++k) {
             int lp, ph;
             pages_get(pre, k, lp, ph);
-            if (ph >= 0 && lp != ex.N - 1) {
+            // the appended token's page too once the inputs are settled
+            if (ph >= 0 && (lp != ex.N - 1 || p.settled)) {
                 if (lane == 0) load_page(k, ph);
                 early |= 1u << k;
             }
@@ -182,12 +185,13 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
         }
     }
 
-    if (p.mode == kModeSparse) {
+    if (p.mode == kModeSparse && !p.settled) {
         // The selection's entries at the speculated positions are loaded together with its count
         // (one round trip); they are the real ones whenever the count is the speculated one.
-        const int lp_real = (lane < nk_spec)
-                                ? p.sel_pages[size_t(b) * p.sel_stride + split * p.items_per_split + warp + lane * WARPS]
-                                : -1;
+        const int lp_real =
+            (lane < nk_spec) ? __ldcg(p.sel_pages + size_t(b) * p.sel_stride + split * p.items_per_split + warp +
+                                      lane * WARPS)
+                             : -1;
         seq_count(p, b, ex);
         i0 = split * p.items_per_split;
         const int i1 = min(i0 + p.items_per_split, ex.count);

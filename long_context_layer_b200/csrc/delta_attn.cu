@@ -517,7 +517,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
                            const int32_t* sel_cnt_in, const int32_t* sel_pages_in, int32_t sel_stride_in,
                            const void* q, const void* k_pool, const void* v_pool, void* o, int32_t* sel_cnt_out,
                            int32_t* sel_pages_out, int32_t sel_stride_out, float* page_scores, void* ws,
-                           size_t ws_bytes, void* stream) {
+                           size_t ws_bytes, void* stream, bool settled = false) {
     delta_status s = check_desc(d);
     if (s != DELTA_OK) return s;
     s = check_pt(pt);
@@ -580,6 +580,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.num_clusters = plan.clusters;
     prm.logits = head_max ? reinterpret_cast<float*>(base + L.logits) : nullptr;
     prm.tickets = reinterpret_cast<int*>(base + L.tickets);
+    prm.settled = (mode == kModeSparse && settled) ? 1 : 0;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     s = launch_decode(d, prm, plan.cluster, plan.wide, pt->batch, st);
@@ -765,6 +766,14 @@ delta_status delta_sparse_attn(const delta_desc* desc, const delta_page_table* p
                                const void* v_pool, void* o, void* workspace, size_t ws_bytes, void* stream) {
     return run_attention(kModeSparse, desc, pt, nullptr, sel_cnt, sel_pages, sel_stride, q, k_pool, v_pool, o, nullptr,
                          nullptr, 0, nullptr, workspace, ws_bytes, stream);
+}
+
+delta_status delta_sparse_attn_settled(const delta_desc* desc, const delta_page_table* pt, const int32_t* sel_cnt,
+                                       const int32_t* sel_pages, int32_t sel_stride, const void* q,
+                                       const void* k_pool, const void* v_pool, void* o, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+    return run_attention(kModeSparse, desc, pt, nullptr, sel_cnt, sel_pages, sel_stride, q, k_pool, v_pool, o, nullptr,
+                         nullptr, 0, nullptr, workspace, ws_bytes, stream, true);
 }
 
 delta_status delta_layer_shift(const delta_page_table* pt, const float* scores_a, const float* scores_b,

@@ -85,6 +85,11 @@ class DeltaStack:
                 scores = self.page_scores[cur] if self.page_scores is not None else None
                 N.select_attn(d, pt, self.sp, q[l], k_pools[l], v_pools[l], out[l], self.sel_cnt[cur],
                               self.sel_pages[cur], self.sel_stride, scores, ws, wb, st)
+            elif l > 0 and self.kinds[l - 1] == SPARSE:
+                # the selection and the appended tokens were final before the previous sparse layer
+                # began (it waited on the selection kernel), so this layer may read them early
+                N.sparse_attn_settled(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l],
+                                      k_pools[l], v_pools[l], out[l], ws, wb, st)
             else:
                 N.sparse_attn(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l], k_pools[l],
                               v_pools[l], out[l], ws, wb, st)

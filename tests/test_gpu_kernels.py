@@ -263,6 +263,14 @@ def test_sparse_attn_matches_oracle(L, G, Hkv, D, dtype, ctx):
         K, V = oracle_kv(dc.case, 0, b)
         ref = O.sparse_attention(dc.case.q(0)[b].astype(np.float64), K, V, sels[b], 16)
         assert_close(out[b], ref, dtype, f"sparse b={b}")
+    # the settled entry (selection read before the wait) gives the same bits; here the previous
+    # kernel of the stream is the sparse call above, so the statement it relies on holds
+    first = dc.out[0].clone()
+    dc.out[0].zero_()
+    L.sparse_attn_settled(desc, pt, sel_cnt, sel_pages, stride, dc.q[0], dc.k_pools[0], dc.v_pools[0], dc.out[0],
+                          ws, nb, stream())
+    ok_flags(L, ws)
+    assert torch.equal(dc.out[0], first)
 
 
 def test_sparse_with_every_page_equals_full(L):
@@ -367,3 +375,25 @@ def test_kv_len_beyond_pages_and_bad_selection_are_flagged(L):
                   stream())
     s, flags = L.read_device_error(ws, stream())
     assert s == 5 and flags & 4
+    L.sparse_attn_settled(desc, pt, sel_cnt, sel_pages, 3, dc.q[0], dc.k_pools[0], dc.v_pools[0], dc.out[0], ws,
+                          nb, stream())
+    s, flags = L.read_device_error(ws, stream())
+    assert s == 5 and flags & 4
+
+
+def test_settled_sparse_flags_a_bad_selection_bf16(L):
+    # the tensor-core kernel reads a settled selection before its wait: bad entries are still
+    # skipped and flagged
+    cfg = make_cfg(7, 2, 128, "bf16", [700])
+    dc = device_case(cfg)
+    desc, pt = make_desc(L, cfg, dc), make_pt(L, dc)
+    ws, nb = workspace(L, desc, dc)
+    sel_pages = torch.tensor([[0, 7, 9999, 43]], dtype=torch.int32, device="cuda")
+    sel_cnt = torch.tensor([4], dtype=torch.int32, device="cuda")
+    L.sparse_attn_settled(desc, pt, sel_cnt, sel_pages, 4, dc.q[0], dc.k_pools[0], dc.v_pools[0], dc.out[0], ws,
+                          nb, stream())
+    s, flags = L.read_device_error(ws, stream())
+    assert s == 5 and flags & 4
+    K, V = oracle_kv(dc.case, 0, 0)
+    ref = O.sparse_attention(dc.case.q(0)[0].astype(np.float64), K, V, [0, 7, 43], 16)
+    assert_close(dc.out[0].float().cpu().numpy()[0], ref, "bf16", "settled, bad entry skipped")
