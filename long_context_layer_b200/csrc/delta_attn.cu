@@ -123,7 +123,12 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wid
     const int warps = wide ? kMmaWideWarps : kWarps;
     const int slots = wide ? sms : sms * split_target_per_sm(dtype, D);
     int s = slots / (units > 0 ? units : 1);
-    const int cap = (items + warps - 1) / warps;
+    // at least one page per warp; 4-warp tensor-core CTAs take at least 7 (two pages for three
+    // warps, one for the fourth): of the plans that give no warp more than one two-page loop
+    // iteration, that one measured fastest on the 8k sparse layers (81 pages: 12 CTAs, against
+    // 16 for one page per warp and 11 for two on every warp)
+    const int per_cta = (!wide && dtype == DELTA_BF16) ? 2 * warps - 1 : warps;
+    const int cap = (items + per_cta - 1) / per_cta;
     if (s > cap) s = cap;
     if (s > kMaxSplits) s = kMaxSplits;
     static int max_splits = -2;
