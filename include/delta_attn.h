@@ -39,10 +39,13 @@
  *     page_scores     [batch][max_pages_per_seq] fp32
  * - Grouped-query attention: query head h reads KV head h / (num_q_heads/num_kv_heads).
  * - Kernels are launched with programmatic dependent launch: a kernel may be scheduled while
- *   the previous kernel of the stream drains, and waits for it before reading q, the pools or a
- *   selection.  The page table and kv_len are treated as inputs of the whole decode step and may
- *   be read before that wait, so a kernel that writes them must complete before the call
- *   (any kernel launched without programmatic dependent launch does).
+ *   the previous kernel of the stream drains, and waits for it before reading q, the page
+ *   holding each sequence's newest token, or a selection (delta_sparse_attn may load pages
+ *   of the selection it finds before the wait, but uses them only if the selection read
+ *   after the wait agrees).  The page table, kv_len and every other pool page are treated as
+ *   inputs of the whole decode step and may be read before that wait, so a kernel that writes
+ *   them must complete before the call (any kernel launched without programmatic dependent
+ *   launch does).  delta_sparse_attn_settled reads everything but q before the wait.
  * - Host-detectable errors return a status and launch nothing.  A launch failure
  *   returns DELTA_ERR_CUDA.  Device-detected errors (a page id outside the pool, a
  *   kv_len beyond the sequence's pages, a selection entry outside the context, a
