@@ -149,7 +149,8 @@ def dist_init():
     if ws > 1:
         import torch.distributed as dist
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        # NCCL on GPUs; the CPU tests of the multi-rank path run the same code over gloo
+        dist.init_process_group(os.environ.get("DELTA_DIST_BACKEND", "nccl"), timeout=timedelta(seconds=120))
         return dist, int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
     return None, 0, 1, 0
 
@@ -166,8 +167,12 @@ def max_over_ranks(dist, x: float, device) -> float:
 def barrier(dist, device):
     import torch
     if dist is not None:
-        dist.barrier(device_ids=[device.index])
-    torch.cuda.synchronize(device)
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+    if device.type == "cuda":
+        torch.cuda.synchronize(device)
 
 
 # ---------------------------------------------------------------------------- accounting
