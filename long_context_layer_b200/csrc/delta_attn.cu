@@ -47,6 +47,10 @@ namespace delta {
 // ------------------------------------------------------------------ host side
 constexpr int kMmaStages = 3;      // tensor-core kernel: stages per warp (8 KB each for D = 128), 2 CTAs/SM
 constexpr int kMmaWideWarps = 8;   // when a cluster per unit fits one CTA per SM: 8-warp CTAs
+constexpr int kMmaShortWarps = 6;  // short page lists: 6 warps with 2 stages each (same shared memory)
+constexpr int kMmaShortStages = 2;
+enum : int { kVarNarrow = 0, kVarWide = 1, kVarShort = 2 };   // tensor-core kernel variants
+constexpr int variant_threads(int v) { return 32 * (v == kVarWide ? kMmaWideWarps : v == kVarShort ? kMmaShortWarps : kWarps); }
 
 struct WsLayout {
     size_t err, tickets, part_ml, part_o, page_lse, split_ml, logits, total;
@@ -99,7 +103,8 @@ int ctas_per_sm(int dtype, int D) {
 // workspace.
 struct SplitPlan {
     int cluster, clusters;
-    bool wide;   // one 8-warp CTA per SM (tensor-core kernel), else 4-warp CTAs, two per SM
+    int variant;   // kVarNarrow: 4-warp CTAs, 3 stages, two per SM; kVarWide: one 8-warp CTA per SM;
+                   // kVarShort: 6-warp CTAs, 2 stages, two per SM (tensor-core kernel)
     int splits() const { return cluster * clusters; }
 };
 
@@ -115,18 +120,18 @@ int split_target_per_sm(int dtype, int D) {
 // About one wave of CTAs, at least one page per warp.  The splits of one (sequence, KV head) form
 // clusters of at most 16 CTAs that merge through distributed shared memory; only long page lists
 // (fit_plan) make several clusters meet in the workspace.
-// The plan of one variant (wide: 8-warp CTAs, one per SM).
-SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wide) {
-    if (items <= 0) return {1, 1, false};
+// The plan of one variant.
+SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, int variant) {
+    if (items <= 0) return {1, 1, kVarNarrow};
+    const bool wide = variant == kVarWide;
     const int sms = device_sm_count();
     const int units = batch * Hkv;
-    const int warps = wide ? kMmaWideWarps : kWarps;
+    const int warps = variant_threads(variant) / 32;
     const int slots = wide ? sms : sms * split_target_per_sm(dtype, D);
     int s = slots / (units > 0 ? units : 1);
-    // at least one page per warp; 4-warp tensor-core CTAs take at least 7 (two pages for three
-    // warps, one for the fourth): of the plans that give no warp more than one two-page loop
-    // iteration, that one measured fastest on the 8k sparse layers (81 pages: 12 CTAs, against
-    // 16 for one page per warp and 11 for two on every warp)
+    // at least one page per warp; 4- and 6-warp tensor-core CTAs take at least 2 * warps - 1
+    // (two pages for all warps but one): of the plans that give no warp more than one two-page
+    // loop iteration, that one measured fastest on the 8k sparse layers (81 pages)
     const int per_cta = (!wide && dtype == DELTA_BF16) ? 2 * warps - 1 : warps;
     const int cap = (items + per_cta - 1) / per_cta;
     if (s > cap) s = cap;
@@ -153,7 +158,7 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, bool wid
     SplitPlan pl;
     pl.cluster = s < 16 ? s : 16;
     pl.clusters = s / pl.cluster;
-    pl.wide = wide;
+    pl.variant = variant;
     return pl;
 }
 
@@ -170,14 +175,21 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
     }
     const bool wide = wide_env && dtype == DELTA_BF16 && int64_t(batch) * Hkv * 16 <= device_sm_count() &&
                       items >= 16 * kMmaWideWarps * 2;
-    return plan_variant(dtype, D, batch, Hkv, items, wide);
+    if (wide) return plan_variant(dtype, D, batch, Hkv, items, kVarWide);
+    // Lists that 4-warp CTAs would cover with at most two pages per warp (a sparse layer of a small
+    // batch): 6 warps with 2 stages each, so more warps share the pages at the same shared memory
+    const SplitPlan narrow = plan_variant(dtype, D, batch, Hkv, items, kVarNarrow);
+    if (dtype == DELTA_BF16 && (items + narrow.splits() - 1) / narrow.splits() <= 2 * kWarps)
+        return plan_variant(dtype, D, batch, Hkv, items, kVarShort);
+    return narrow;
 }
 
 // Most splits any launch on page lists of at most max_pages can get (workspace bound): both
 // variants' split counts grow with the page count.
 int max_splits_for(int dtype, int D, int batch, int Hkv, int max_pages) {
-    const int a = plan_variant(dtype, D, batch, Hkv, max_pages, false).splits();
-    const int b = plan_variant(dtype, D, batch, Hkv, max_pages, true).splits();
+    // (a short-list plan never has more splits than the 4-warp plan of the same list)
+    const int a = plan_variant(dtype, D, batch, Hkv, max_pages, kVarNarrow).splits();
+    const int b = plan_variant(dtype, D, batch, Hkv, max_pages, kVarWide).splits();
     return a > b ? a : b;
 }
 
@@ -275,10 +287,14 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const delta_desc* d) {
 
 // ---- kernel selection and cluster occupancy
 template <int D, int G>
-const void* mma_ptr(bool wide, size_t* smem) {
-    if (wide) {
+const void* mma_ptr(int variant, size_t* smem) {
+    if (variant == kVarWide) {
         *smem = MmaSmem<D, kMmaStages, kMmaWideWarps>::kBytes;
         return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStages, kMmaWideWarps>);
+    }
+    if (variant == kVarShort) {
+        *smem = MmaSmem<D, kMmaShortStages, kMmaShortWarps>::kBytes;
+        return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaShortStages, kMmaShortWarps>);
     }
     *smem = MmaSmem<D, kMmaStages>::kBytes;
     return reinterpret_cast<const void*>(decode_mma_kernel<D, G, kMmaStages, kWarps>);
@@ -301,14 +317,14 @@ const void* simt_ptr(size_t* smem) {
         case 8: return CALL(8); \
         default: return nullptr; \
     }
-const void* decode_ptr(int dtype, int D, int G, bool wide, size_t* smem) {
+const void* decode_ptr(int dtype, int D, int G, int variant, size_t* smem) {
     if (dtype == DELTA_BF16) {
         if (D == 128) {
-#define CALL(g) mma_ptr<128, g>(wide, smem)
+#define CALL(g) mma_ptr<128, g>(variant, smem)
             DELTA_G_PTR(G, CALL)
 #undef CALL
         }
-#define CALL(g) mma_ptr<64, g>(wide, smem)
+#define CALL(g) mma_ptr<64, g>(variant, smem)
         DELTA_G_PTR(G, CALL)
 #undef CALL
     }
@@ -398,9 +414,9 @@ SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) 
         cand.clusters = s / c < max_clusters ? s / c : max_clusters;
         if (cand.clusters < 1) continue;
         size_t smem = 0;
-        const void* fn = decode_ptr(dtype, D, G, cand.wide, &smem);
+        const void* fn = decode_ptr(dtype, D, G, cand.variant, &smem);
         if (fn == nullptr) return pl;
-        const int maxc = max_active_clusters(fn, smem, c, cand.wide ? kMmaWideWarps * 32 : kThreads);
+        const int maxc = max_active_clusters(fn, smem, c, dtype == DELTA_BF16 ? variant_threads(cand.variant) : kThreads);
         if (int64_t(units) * cand.clusters > maxc) {
             cand.clusters = maxc / units;
             if (cand.clusters < 1) continue;
@@ -414,7 +430,7 @@ SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) 
     if (best_ctas < 0) {   // more units than resident clusters even at size 1: several waves
         best.cluster = 1;
         best.clusters = 1;
-        best.wide = false;
+        best.variant = kVarNarrow;
     }
     return best;
 }
@@ -469,11 +485,15 @@ delta_status launch_simt_g(const DecodeParams& prm, int cluster, int batch, int 
 
 template <int D, int G>
 delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const CUtensorMap& mv, int cluster,
-                          bool wide, int batch, int Hkv, cudaStream_t st) {
-    if (wide)
+                          int variant, int batch, int Hkv, cudaStream_t st) {
+    if (variant == kVarWide)
         return launch_clustered(decode_mma_kernel<D, G, kMmaStages, kMmaWideWarps>,
                                 MmaSmem<D, kMmaStages, kMmaWideWarps>::kBytes, kMmaWideWarps * 32, prm, cluster, batch,
                                 Hkv, st, mk, mv);
+    if (variant == kVarShort)
+        return launch_clustered(decode_mma_kernel<D, G, kMmaShortStages, kMmaShortWarps>,
+                                MmaSmem<D, kMmaShortStages, kMmaShortWarps>::kBytes, kMmaShortWarps * 32, prm, cluster,
+                                batch, Hkv, st, mk, mv);
     return launch_clustered(decode_mma_kernel<D, G, kMmaStages, kWarps>, MmaSmem<D, kMmaStages>::kBytes, kThreads, prm,
                             cluster, batch, Hkv, st, mk, mv);
 }
@@ -491,18 +511,18 @@ delta_status launch_mma_g(const DecodeParams& prm, const CUtensorMap& mk, const 
         default: return DELTA_ERR_UNSUPPORTED; \
     }
 
-delta_status launch_decode(const delta_desc* d, const DecodeParams& prm, int cluster, bool wide, int batch,
+delta_status launch_decode(const delta_desc* d, const DecodeParams& prm, int cluster, int variant, int batch,
                            cudaStream_t st) {
     const int Hkv = d->num_kv_heads, G = d->num_q_heads / Hkv;
     if (d->dtype == DELTA_BF16) {
         CUtensorMap mk, mv;
         if (!make_pool_map(&mk, prm.k_pool, d) || !make_pool_map(&mv, prm.v_pool, d)) return DELTA_ERR_CUDA;
         if (d->head_dim == 128) {
-#define CALL(g) launch_mma_g<128, g>(prm, mk, mv, cluster, wide, batch, Hkv, st)
+#define CALL(g) launch_mma_g<128, g>(prm, mk, mv, cluster, variant, batch, Hkv, st)
             DELTA_G_SWITCH(G, CALL)
 #undef CALL
         } else {
-#define CALL(g) launch_mma_g<64, g>(prm, mk, mv, cluster, wide, batch, Hkv, st)
+#define CALL(g) launch_mma_g<64, g>(prm, mk, mv, cluster, variant, batch, Hkv, st)
             DELTA_G_SWITCH(G, CALL)
 #undef CALL
         }
@@ -588,7 +608,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.settled = (mode == kModeSparse && settled) ? 1 : 0;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    s = launch_decode(d, prm, plan.cluster, plan.wide, pt->batch, st);
+    s = launch_decode(d, prm, plan.cluster, plan.variant, pt->batch, st);
     if (s != DELTA_OK || mode != kModeDelta) return s;
 
     SelectParams sp2{};
