@@ -223,7 +223,6 @@ struct SeqExtent {
     int N;                  // pages
     int pbeg;               // first entry of the sequence in page_indices
     int count;              // items to attend: N, or the selection length
-    const int32_t* table;   // the sequence's page-table row staged in shared memory, or null
 };
 
 // QUIET: a speculative lookup (before the wait, for an L2 prefetch only) that raises no flags.
@@ -243,7 +242,7 @@ __device__ __forceinline__ void fetch_pages(const P& p, const SeqExtent& ex, int
         lp = -1;
         return;
     }
-    const int64_t x = ex.table != nullptr ? ex.table[lp] : p.indices[ex.pbeg + lp];
+    const int64_t x = p.indices[ex.pbeg + lp];
     if (x < 0 || x >= p.num_phys_pages) {
         if (!QUIET) atomicOr(p.err, kErrPage);
         return;
@@ -294,7 +293,6 @@ __device__ __forceinline__ SeqExtent seq_extent(const P& p, int b) {
     ex.n = n;
     ex.N = (n + kPage - 1) / kPage;
     ex.count = ex.N;
-    ex.table = nullptr;
     return ex;
 }
 
@@ -422,7 +420,7 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
             acc = fmaf(w, recv[j * chunk + (e - e0)], acc);
         }
         if (nC == 1) {
-            out[(size_t(b) * Hq + h0 + h) * D + d] = Elem<T>::from_f(M == -INFINITY ? 0.f : acc / L);
+            out[(size_t(b) * Hq + h0 + h) * D + d] = Elem<T>::from_f(M == -INFINITY ? 0.f : __fdividef(acc, L));
         } else {
             const size_t row = (size_t(b) * Hq + h0 + h) * nC + cidx;
             p.part_o[row * D + d] = acc;

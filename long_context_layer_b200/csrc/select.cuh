@@ -53,8 +53,7 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& 
     __syncthreads();
     const int res = warp_sums[warp] + incl - x;
     total = warp_sums[32];
-    __syncthreads();
-    return res;
+    return res;   // warp_sums is not written again: no trailing barrier
 }
 
 // Shared-memory plan of the selection cluster (dynamic): keys of this CTA's pages, the keys of the
@@ -378,10 +377,14 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const Sele
     const int packed = block_exclusive_scan(eq_cnt | (gtf_cnt << 16), warp_sums, tot_loc);
     const int eq_rank_loc = packed & 0xffff, gtf_rank_loc = packed >> 16;
     const int eq_tot_loc = tot_loc & 0xffff, gtf_tot_loc = tot_loc >> 16;
-    if (tid < C) cluster.map_shared_rank(recv_cnt, tid)[rank] = make_int2(eq_tot_loc, gtf_tot_loc);
-    cluster_barrier();
     int eq_cum = 0, eq_before = 0, sel_before = 0, total = 0;
-    for (int j = 0; j < C; ++j) {
+    if (C == 1) {   // one CTA: its own totals
+        total = gtf_tot_loc + min(int(need_eq), eq_tot_loc);
+    } else {
+        if (tid < C) cluster.map_shared_rank(recv_cnt, tid)[rank] = make_int2(eq_tot_loc, gtf_tot_loc);
+        cluster_barrier();
+    }
+    for (int j = 0; j < C && C > 1; ++j) {
         const int2 v = recv_cnt[j];
         const int taken = min(max(int(need_eq) - eq_cum, 0), v.x);   // T-valued pages of CTA j that are kept
         if (j < rank) {
