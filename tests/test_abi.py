@@ -122,3 +122,19 @@ def test_empty_batch_is_a_no_op(L):
     pt = L.DeltaPageTable(None, None, None, 0, 0)
     assert L.full_attn(d, pt, None, None, None, None, None, 0, 0, check=False) == 0
     assert L.kv_append(d, pt, None, None, None, None, 0, check=False) == 0
+
+
+def test_stack_placement_rule_matches_the_oracle():
+    # the product's delta-layer placement (restated in stack.py) equals the oracle's on random shifts,
+    # ties included
+    import numpy as np
+    from oracle import delta_oracle as O
+    from long_context_layer_b200.stack import choose_delta_layers
+    r = np.random.default_rng(7)
+    for _ in range(200):
+        L = int(r.integers(4, 49))
+        shift = np.round(r.random(L), 1)          # coarse values: many exact ties
+        shift[:2] = 0.0
+        count = int(r.integers(1, 6))
+        gap = int(r.integers(1, 4))
+        assert choose_delta_layers(shift, count, min_gap=gap) == O.choose_delta_layers(shift, count, min_gap=gap)

@@ -293,7 +293,7 @@ def test_layer_shift_matches_library_cosine():
 def test_choose_delta_layers_rules():
     shift = np.array([0, 0, 0.1, 0.9, 0.85, 0.2, 0.7, 0.1, 0.8])
     assert O.choose_delta_layers(shift, 1) == [2]
-    # 3 is the largest shift but is adjacent to 2; 8 and 6 follow (4 too close to 3? 3 is not chosen)
+    # by shift: 3 (one layer from 2: skipped), 4, 8, then 6
     assert O.choose_delta_layers(shift, 3, min_gap=2) == [2, 4, 8]
     assert O.choose_delta_layers(shift, 4, min_gap=2) == [2, 4, 6, 8]
     assert O.choose_delta_layers(shift, 3, min_gap=1) == [2, 3, 4]
