@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
     ap.add_argument("--print-source-hash", action="store_true", help="print the kernel-source hash and exit")
     ap.add_argument("--drift-checks", type=int, default=10, help="oracle selection checks along a trajectory")
+    ap.add_argument("--reduce", choices=["sum", "max"], default="sum",
+                    help="head aggregation of the page score: sum (default) or the page's max rule")
     ap.add_argument("--delta-sweep", type=str, default="",
                     help="comma list of delta-layer counts: time the step for each (spread placement)")
     return ap.parse_args()
@@ -404,9 +406,10 @@ def run_ours(args):
     case = Case(cfg)
     dc = DeviceCase(case, device=device, prefill="append")
     kinds = cfg.layer_kinds()
+    reduce = NAT.DELTA_HEAD_MAX if args.reduce == "max" else NAT.DELTA_HEAD_SUM
     mk = lambda kk: DeltaStack(kk, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr, dc.indices,
                                dc.kv_len, case.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages,
-                               cfg.sink_tokens, cfg.recency_tokens)
+                               cfg.sink_tokens, cfg.recency_tokens, reduce=reduce)
     delta_stack = mk(kinds)
     full_stack = mk(["full"] * cfg.num_layers)
     args_step = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
@@ -560,7 +563,7 @@ def run_ours(args):
                        "batch": cfg.batch, "context": int(case.n.max()), "page_size": cfg.page_size,
                        "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
                        "recency_tokens": cfg.recency_tokens, "l2": "flushed before every timed replay (2xL2 write, then 2xL2 read)",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}", "score": f"head {args.reduce}"},
             "full_stack_us": round(us_full, 3),
             "speedup_vs_full_stack": round(us_full / us_delta, 3),
             "attended_token_reduction": round(tok_full / tok_delta, 3),
