@@ -628,9 +628,11 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     sp2.page_scores = page_scores;
     sp2.logits = prm.logits;
     sp2.err = prm.err;
-    // one cluster of C CTAs per sequence, about 16K page partials per CTA
+    // one cluster of C CTAs per sequence, about 16K page terms per CTA; HEAD_MAX scores every
+    // token of every head (a warp per page), so there a CTA takes about one page per warp
     const int maxp = pt->max_pages_per_seq;
-    int C = int((int64_t(Hq) * maxp + 16383) / 16384);
+    int C = head_max ? (maxp + kSelectThreads / 32 - 1) / (kSelectThreads / 32)
+                     : int((int64_t(Hq) * maxp + 16383) / 16384);
     C = C < 1 ? 1 : (C > 16 ? 16 : C);
     const int chunk = (maxp + C - 1) / C;
     const SelectSmem SL{chunk, C};
