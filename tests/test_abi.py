@@ -113,6 +113,10 @@ def test_sparse_and_append_arguments_rejected(L):
     ws = L.workspace_size(d, 1, 512)
     assert L.sparse_attn(d, _pt(L), None, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 0, check=False) == 1
     assert L.sparse_attn(d, _pt(L), FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 0, check=False) == 1
+    assert L.sparse_attn_settled(d, _pt(L), None, FAKE, 10, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 0, check=False) == 1
+    assert L.sparse_attn_settled(d, _pt(L), FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 0, check=False) == 1
+    assert L.sparse_attn_settled(d, _pt(L), FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, None, ws, 0, check=False) == 3
+    assert L.layer_shift(_pt(L), None, FAKE, FAKE, 0, check=False) == 1
     assert L.kv_append(d, _pt(L), None, FAKE, FAKE, FAKE, 0, check=False) == 1
     assert L.kv_append(_desc(L, head_dim=80), _pt(L), FAKE, FAKE, FAKE, FAKE, 0, check=False) == 2
 
