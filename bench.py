@@ -522,24 +522,32 @@ def run_ours(args):
     achieved_sparse = alg_sparse / (us_sparse_launch * 1e-6) / 1e9
     n_sparse = kinds.count("sparse")
 
-    # -- end to end through the public API: pinned host inputs in, outputs out, every step
-    q_h = dc.q.cpu().pin_memory()
-    kn_h, vn_h = dc.k_new.cpu().pin_memory(), dc.v_new.cpu().pin_memory()
+    # -- end to end through the public API: every step the step's inputs (q, k_new, v_new) come
+    #    from one pinned host staging buffer in one copy, the step runs (the same calls, captured in
+    #    a graph over views of the device staging buffer) and every layer's output goes back to
+    #    pinned host memory
+    nq, nk = dc.q.numel(), dc.k_new.numel()
+    in_h = torch.cat([dc.q.reshape(-1), dc.k_new.reshape(-1), dc.v_new.reshape(-1)]).cpu().pin_memory()
+    in_d = torch.empty_like(in_h, device=device)
+    in_d.copy_(in_h)
+    q_v = in_d[:nq].view_as(dc.q)
+    kn_v = in_d[nq:nq + nk].view_as(dc.k_new)
+    vn_v = in_d[nq + nk:].view_as(dc.v_new)
     out_h = torch.empty_like(dc.out, device="cpu").pin_memory()
-    sel_h = torch.empty_like(delta_stack.sel_pages, device="cpu").pin_memory()
+    e2e_stack = mk(kinds)
+    g_e2e = e2e_stack.capture(q_v, kn_v, vn_v, dc.k_pools, dc.v_pools, dc.out)
 
     def e2e_step():
-        dc.q.copy_(q_h, non_blocking=True)
-        dc.k_new.copy_(kn_h, non_blocking=True)
-        dc.v_new.copy_(vn_h, non_blocking=True)
-        g_delta.replay()
+        in_d.copy_(in_h, non_blocking=True)
+        g_e2e.replay()
         out_h.copy_(dc.out, non_blocking=True)
-        sel_h.copy_(delta_stack.sel_pages, non_blocking=True)
 
     t_e2e = timed(e2e_step, args.steps, 3)
     us_e2e = max_over_ranks(dist, statistics.mean(t_e2e), device)
-    h2d = (q_h.numel() + kn_h.numel() + vn_h.numel()) * e
-    d2h = out_h.numel() * e + sel_h.numel() * 4
+    h2d = in_h.numel() * e
+    d2h = out_h.numel() * e
+    del g_e2e
+    e2e_stack.graph = None
 
     tok_delta, tok_full, _, _ = attended_tokens(cfg, case)
     cpu = None
