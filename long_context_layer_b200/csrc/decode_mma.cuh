@@ -1,6 +1,6 @@
 // Tensor-core split-KV decode kernel for bf16 storage (included by delta_attn.cu only).
 //
-// One CTA = (split, KV head, sequence); each of its 4 warps streams whole pages.  A page of one
+// One CTA = (split, KV head, sequence); each of its WARPS warps (4, 6 or 8) streams whole pages.  A page of one
 // KV head (16 tokens x D) of K and of V arrives in the warp's shared-memory stage through 2-D
 // TMA tensor copies (cp.async.bulk.tensor, 64-column boxes, 128-byte swizzle) completing on an
 // mbarrier.  Per page:
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
     }
 
     // ---- this warp's state into its own stage area (all of its copies have landed and no other
-    // warp touches that area), one barrier, then the merge of the 4 warps and of the splits
+    // warp touches that area), one barrier, then the merge of the CTA's warps and of the splits
     __syncwarp();
     // rows padded by 4 floats: the four lanes of a column group (t4) store to different banks
     constexpr int kRow = D + 4;

@@ -5,26 +5,27 @@
 // delta-layers run full attention and score 16-token KV pages, sparse layers attend only to
 // the selected pages; the paged KV cache is kept in full.
 //
-// Kernels (all launched on the caller's stream, none synchronises the host):
-//   kv_append_kernel      one (sequence, KV head) per CTA, 16-byte vector copies.
-//   decode_kernel         split-KV online-softmax decode.  Grid (split, KV head, sequence).
-//                         Each of the 4 warps streams whole pages (K and V of one KV head,
-//                         2*16*D elements) from HBM into its own shared-memory ring with
-//                         1-D TMA bulk copies (cp.async.bulk + mbarrier transaction counts)
-//                         and packs the G query heads of the group against them: a half-warp
-//                         owns 8 tokens of a page, a lane owns D/16 dimensions; partial dot
-//                         products are reduce-scattered across the half-warp so each lane
-//                         ends with one (token, head) logit.  The delta variant also writes
-//                         each page's (max logit, sum exp) per query head.  The sparse
-//                         variant walks the selected page list instead of 0..N-1.
-//                         The split partials of a (sequence, KV head) are merged by whichever
-//                         of its CTAs arrives last (an atomic ticket; no CTA ever waits), which
-//                         writes o and, for delta-layers, each head's (max, sum-exp) pair.
-//   score_select_kernel   one thread-block cluster per sequence: page score = sum over heads of
-//                         2^(m_hp - M_h) l_hp / L_h, then an MSB-first 4x8-bit radix select of
-//                         the k-th largest candidate score with shared-memory histograms,
-//                         lower-index tie-break by a block prefix scan, union with sink and
-//                         recency pages, ascending compaction.
+// Kernels (all launched on the caller's stream with programmatic dependent launch, none
+// synchronises the host):
+//   kv_append_kernel,     the current token's k, v into its page slot: one (sequence, KV head)
+//   kv_append_layers_     per CTA (and per layer), 16-byte vector copies.
+//     kernel
+//   decode_mma_kernel     bf16 split-KV online-softmax decode on the tensor cores (mma.sync,
+//                         decode_mma.cuh).  Grid (split, KV head, sequence) in thread-block
+//                         clusters; each warp streams whole pages (K and V of one KV head) into
+//                         its own shared-memory ring with 2-D TMA tensor copies.  Delta-layers
+//                         also write each (head, page)'s log2-sum-exp and each split's per-head
+//                         state; sparse layers walk the selected page list.  Splits merge by
+//                         pushing their partials into the owning CTA of the cluster (st.async
+//                         on its mbarrier); several clusters of one unit meet in the workspace,
+//                         merged by whichever CTA arrives last (an atomic ticket; no CTA waits).
+//   decode_kernel         the fp32 counterpart on the CUDA cores (decode_simt.cuh), same merge.
+//   score_select_kernel   one thread-block cluster per sequence (select.cuh): page score = sum
+//                         over heads of 2^(lse_hp - c_h), c_h from the splits' states; the k-th
+//                         largest candidate by a bucket histogram and an exact in-bucket rank
+//                         (one CTA) or an MSB-first radix select (cluster); lower-index tie-break,
+//                         union with sink and recency pages, ascending compaction.
+//   layer_shift_kernel    1 - cos between two layers' page-score vectors (calibration metric).
 //
 // Logits are carried in base 2 (q is pre-scaled by sm_scale*log2(e)) so every exponential is
 // one exp2.  No floating-point atomics are used: results are deterministic run to run.
@@ -170,7 +171,7 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
     // CTAs, two per SM, so the next layer's CTAs find room beside them and start their loads.
     static int wide_env = -1;
     if (wide_env < 0) {
-        const char* e = getenv("DELTA_WIDE");   // tuning override for sweeps (0: always 4 warps)
+        const char* e = getenv("DELTA_WIDE");   // tuning override for sweeps (0: no 8-warp CTAs)
         wide_env = (e != nullptr && atoi(e) == 0) ? 0 : 1;
     }
     const bool wide = wide_env && dtype == DELTA_BF16 && int64_t(batch) * Hkv * 16 <= device_sm_count() &&
