@@ -563,8 +563,11 @@ def run_ours(args):
     launches = delta_stack.launches_per_step() * args.steps
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(us_delta, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(us_delta / 1000, 6), "higher_is_better": False,
+            # whole job: N replicas each finish a decode step in us_delta (slowest rank), so the job
+            # spends us_delta / N per decode step; ms_per_step is one step iteration of the job
+            "metric": METRIC, "value": round(us_delta / world, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us_delta / 1000, 6),
+            "replica_step_us": round(us_delta, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "layers": cfg.num_layers, "delta_layers": list(cfg.delta_layers),
                        "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
@@ -595,7 +598,8 @@ def run_ours(args):
                                     "single_call_frac": round(achieved_single / peak, 4),
                                     "traffic": profiled_traffic(cfg.name, "full_layer")},
             "breakdown_us_per_call": breakdown,
-            "e2e": {"value": round(us_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": round(us_e2e / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
