@@ -45,3 +45,12 @@ def test_attended_tokens_match_the_oracle_selection():
         kinds = cfg.layer_kinds()
         assert full_tok_stack == len(kinds) * n
         assert delta_tok == kinds.count("sparse") * sparse_tok + (len(kinds) - kinds.count("sparse")) * n
+
+
+def test_sweep_placement_spreads_delta_layers_from_layer_2():
+    import bench
+    for L in (28, 32, 48):
+        for m in range(1, L - 1):
+            pl = bench.delta_placement(L, m)
+            assert pl[0] == 2 and len(pl) == m and pl == sorted(set(pl)) and pl[-1] < L
+        assert bench.delta_placement(L, L - 2) == list(range(2, L))   # every layer from 2: the full stack
