@@ -20,8 +20,12 @@
  * --------------------------------
  * - Every pointer argument is DEVICE memory owned by the caller, except the
  *   descriptor structs themselves, which are read on the host during the call.
- *   The library allocates nothing and keeps no state between calls beyond a
- *   cached per-device attribute query.
+ *   The library allocates nothing and reads no environment variable.  Between
+ *   calls it keeps only per-device caches filled on first use and never changed
+ *   afterwards (SM count, kernel attributes it set, cluster occupancy, the driver's
+ *   tensor-map encoder, the address of delta_full_attn_noalloc's scratch array),
+ *   guarded by a mutex; a device reset (cudaDeviceReset) invalidates them, so
+ *   reload the library after one.
  * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *   Every call only enqueues work: none synchronises the host, so every call can
  *   be captured in a CUDA graph.  Outputs are valid once the stream reaches them.

@@ -36,7 +36,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
-#include <stdlib.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -67,8 +68,16 @@ int current_device() {
     return dev;
 }
 
+// Guards the per-device caches below (SM count, kernel attributes, cluster occupancy, the tensor-map
+// encoder and the scratch array's address): first calls from several host threads may race.
+std::recursive_mutex& cache_mutex() {
+    static std::recursive_mutex mu;
+    return mu;
+}
+
 int device_sm_count() {
     static int cache[64] = {0};
+    std::lock_guard<std::recursive_mutex> lock(cache_mutex());
     const int dev = current_device();
     if (dev < 0) return 148;
     if (cache[dev] == 0) {
@@ -109,13 +118,31 @@ struct SplitPlan {
     int splits() const { return cluster * clusters; }
 };
 
+// Split-plan constants (compile-time; a sweep rebuilds the library with -D overrides).
+#ifndef DELTA_CTAS_PER_SM
+#define DELTA_CTAS_PER_SM 0          // 0: as many CTAs per SM as shared memory allows
+#endif
+#ifndef DELTA_MAX_SPLITS
+#define DELTA_MAX_SPLITS 0           // 0: no cap beyond kMaxSplits
+#endif
+#ifndef DELTA_MAX_WIDE_SPLITS
+#define DELTA_MAX_WIDE_SPLITS 0      // 0: no extra cap on 8-warp plans
+#endif
+#ifndef DELTA_MAX_NARROW_SPLITS
+#define DELTA_MAX_NARROW_SPLITS 0    // 0: no extra cap on 4- and 6-warp plans
+#endif
+#ifndef DELTA_WIDE
+#define DELTA_WIDE 1                 // 0: never use 8-warp CTAs
+#endif
+#ifndef DELTA_PAGES_PER_CLUSTER
+#define DELTA_PAGES_PER_CLUSTER 256  // pages each cluster must get before a unit uses several
+#endif
+#ifndef DELTA_ONE_CLUSTER_PAGES
+#define DELTA_ONE_CLUSTER_PAGES 512  // up to this many pages per unit, one cluster
+#endif
+
 int split_target_per_sm(int dtype, int D) {
-    static int override_ = -2;
-    if (override_ == -2) {
-        const char* e = getenv("DELTA_CTAS_PER_SM");   // tuning override for sweeps
-        override_ = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
-    }
-    return override_ > 0 ? override_ : ctas_per_sm(dtype, D);
+    return DELTA_CTAS_PER_SM > 0 ? DELTA_CTAS_PER_SM : ctas_per_sm(dtype, D);
 }
 
 // About one wave of CTAs, at least one page per warp.  The splits of one (sequence, KV head) form
@@ -137,24 +164,9 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, int vari
     const int cap = (items + per_cta - 1) / per_cta;
     if (s > cap) s = cap;
     if (s > kMaxSplits) s = kMaxSplits;
-    static int max_splits = -2;
-    if (max_splits == -2) {
-        const char* e = getenv("DELTA_MAX_SPLITS");   // tuning override for sweeps
-        max_splits = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
-    }
-    if (max_splits > 0 && s > max_splits) s = max_splits;
-    static int max_wide = -2;
-    if (max_wide == -2) {
-        const char* e = getenv("DELTA_MAX_WIDE_SPLITS");   // tuning override for sweeps
-        max_wide = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
-    }
-    if (wide && max_wide > 0 && s > max_wide) s = max_wide;
-    static int max_narrow = -2;
-    if (max_narrow == -2) {
-        const char* e = getenv("DELTA_MAX_NARROW_SPLITS");   // tuning override for sweeps
-        max_narrow = (e != nullptr && atoi(e) > 0) ? atoi(e) : -1;
-    }
-    if (!wide && max_narrow > 0 && s > max_narrow) s = max_narrow;
+    if (DELTA_MAX_SPLITS > 0 && s > DELTA_MAX_SPLITS) s = DELTA_MAX_SPLITS;
+    if (wide && DELTA_MAX_WIDE_SPLITS > 0 && s > DELTA_MAX_WIDE_SPLITS) s = DELTA_MAX_WIDE_SPLITS;
+    if (!wide && DELTA_MAX_NARROW_SPLITS > 0 && s > DELTA_MAX_NARROW_SPLITS) s = DELTA_MAX_NARROW_SPLITS;
     if (s < 1) s = 1;
     SplitPlan pl;
     pl.cluster = s < 16 ? s : 16;
@@ -169,12 +181,7 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
     // of a 4-warp CTA's warp (the per-warp chain of dependent MMAs, exponentials and shuffles,
     // not the memory system, bounds such layers).  Short page lists (sparse layers) keep 4-warp
     // CTAs, two per SM, so the next layer's CTAs find room beside them and start their loads.
-    static int wide_env = -1;
-    if (wide_env < 0) {
-        const char* e = getenv("DELTA_WIDE");   // tuning override for sweeps (0: no 8-warp CTAs)
-        wide_env = (e != nullptr && atoi(e) == 0) ? 0 : 1;
-    }
-    const bool wide = wide_env && dtype == DELTA_BF16 && int64_t(batch) * Hkv * 16 <= device_sm_count() &&
+    const bool wide = DELTA_WIDE && dtype == DELTA_BF16 && int64_t(batch) * Hkv * 16 <= device_sm_count() &&
                       items >= 16 * kMmaWideWarps * 2;
     if (wide) return plan_variant(dtype, D, batch, Hkv, items, kVarWide);
     // Lists that 4-warp CTAs would cover with at most two pages per warp (a sparse layer of a small
@@ -242,19 +249,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 delta_status launch_status() { return cudaPeekAtLastError() == cudaSuccess ? DELTA_OK : DELTA_ERR_CUDA; }
 
-// Raise a kernel's dynamic shared-memory limit once per device.
-template <typename K>
-bool set_smem_once(K kern, size_t bytes, int* configured) {
-    const int dev = current_device();
-    if (dev < 0) return false;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess)
-            return false;
-        configured[dev] = 1;
-    }
-    return true;
-}
-
 // ---- tensor maps (driver entry point resolved through the runtime; no libcuda link needed)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -262,6 +256,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
+    std::lock_guard<std::recursive_mutex> lock(cache_mutex());
     if (fn == nullptr) {
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -343,6 +338,7 @@ const void* decode_ptr(int dtype, int D, int G, int variant, size_t* smem) {
 bool configure_kernel(const void* func, size_t smem) {
     constexpr int kSlots = 256;
     static const void* done_fn[64][kSlots];
+    std::lock_guard<std::recursive_mutex> lock(cache_mutex());
     const int dev = current_device();
     if (dev < 0) return false;
     int i = 0;
@@ -360,6 +356,7 @@ int max_active_clusters(const void* func, size_t smem, int cluster, int threads)
     constexpr int kSlots = 512;
     struct Entry { const void* fn; int cluster; int n; };
     static Entry cache[64][kSlots];
+    std::lock_guard<std::recursive_mutex> lock(cache_mutex());
     const int dev = current_device();
     if (dev < 0) return 1;
     int i = 0;
@@ -395,17 +392,8 @@ SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) 
     const int s = pl.splits();
     // Clusters meet through the workspace only when each gets at least 256 pages (and the unit has
     // more than 512): below that the cross-cluster merge costs more than the extra CTAs gain.
-    static int per_cluster = -1;
-    if (per_cluster < 0) {
-        const char* e = getenv("DELTA_PAGES_PER_CLUSTER");   // tuning override for sweeps
-        per_cluster = (e != nullptr && atoi(e) > 0) ? atoi(e) : 256;
-    }
     // Up to 512 pages per (sequence, KV head) one cluster is faster (measured on the 8k stack).
-    static int one_cluster = -1;
-    if (one_cluster < 0) {
-        const char* e = getenv("DELTA_ONE_CLUSTER_PAGES");   // tuning override for sweeps
-        one_cluster = (e != nullptr && atoi(e) >= 0) ? atoi(e) : 512;
-    }
+    constexpr int per_cluster = DELTA_PAGES_PER_CLUSTER, one_cluster = DELTA_ONE_CLUSTER_PAGES;
     const int max_clusters = (items <= one_cluster || items / per_cluster < 1) ? 1 : items / per_cluster;
     SplitPlan best = pl;
     int best_ctas = -1;
@@ -670,6 +658,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kStaticScratchB
 // host code the array's name only stands for the symbol; the kernel must get this address.
 unsigned char* noalloc_scratch() {
     static unsigned char* addr[64] = {nullptr};
+    std::lock_guard<std::recursive_mutex> lock(cache_mutex());
     const int dev = current_device();
     if (dev < 0) return nullptr;
     if (addr[dev] == nullptr) {
