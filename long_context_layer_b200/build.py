@@ -4,8 +4,9 @@
 
 (Run it by path: importing the package loads the library this script builds.)
 
-Produces long_context_layer_b200/libdelta_attn.so (the C ABI of include/delta_attn.h) and
-synth/libsynth_fill.so (the device-side input generator used by tests and the benchmark).
+Produces long_context_layer_b200/libdelta_attn.so (the C ABI of include/delta_attn.h),
+synth/libsynth_fill.so (the device-side input generator used by tests and the benchmark) and
+synth/libsynth_host.so (the same generator on the host, for fast oracle inputs).
 """
 from __future__ import annotations
 
@@ -25,6 +26,10 @@ TARGETS = [
     (os.path.join(ROOT, "synth", "csrc", "synth_fill.cu"),
      os.path.join(ROOT, "synth", "libsynth_fill.so"), []),
 ]
+# host (CPU) libraries built with gcc: the input generator's host copy
+HOST_TARGETS = [
+    (os.path.join(ROOT, "synth", "csrc", "synth_host.c"), os.path.join(ROOT, "synth", "libsynth_host.so")),
+]
 
 
 def nvcc() -> str:
@@ -43,6 +48,14 @@ def build(force: bool = False, verbose: bool = False) -> list:
         if not force and os.path.exists(out) and os.path.getmtime(out) >= max(os.path.getmtime(d) for d in deps):
             continue
         cmd = [nvcc()] + ARCH + COMMON + extra + [src, "-o", out]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.run(cmd, check=True)
+        built.append(out)
+    for src, out in HOST_TARGETS:
+        if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+            continue
+        cmd = ["gcc", "-O3", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", src, "-o", out]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.run(cmd, check=True)

@@ -165,6 +165,12 @@ __device__ __forceinline__ void load_row<float, 4>(const float* p, float (&x)[4]
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
 }
 
+// Order-preserving 32-bit key of a float (larger float, larger key).
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 __host__ __device__ constexpr int pad_group(int g) { return g <= 1 ? 1 : g <= 2 ? 2 : g <= 4 ? 4 : 8; }
 
 // ------------------------------------------------------------------ decode kernel
@@ -198,6 +204,18 @@ struct DecodeParams {
     float* logits;          // [B][Hq][max_pages*16] base-2 logits (delta-layers in HEAD_MAX mode), else null
     int* tickets;     // [B][Hkv] arrival counters of the split CTAs, zero between launches
     int* err;
+    // Delta-layers scoring with HEAD_SUM: the page selection runs at the end of the decode kernel
+    // (select_tail.cuh) instead of in a separate launch.
+    int32_t fuse_select;
+    int32_t budget_pages, sink_tokens, recency_tokens;
+    int32_t* sel_cnt_out;     // [B]
+    int32_t* sel_pages_out;   // [B][sel_stride_out]
+    int32_t sel_stride_out;
+    float* page_scores;       // [B][max_pages] or null
+    float* unit_scores;       // [B][Hkv][max_pages] each (sequence, KV head) unit's share of the page scores
+    uint32_t* keys;           // [B][max_pages] order keys of the page scores (when shared memory is short)
+    int* unit_tickets;        // [B][Hkv] CTAs of a unit that finished, zero between launches
+    int* seq_tickets;         // [B] units of a sequence that finished, zero between launches
 };
 
 

@@ -16,6 +16,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "select_tail.cuh"
 
 namespace delta {
 
@@ -444,6 +445,8 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
     merge_epilogue<__nv_bfloat16, D, G, WARPS, WARPS * 32, kRow>(
         p, smem, mo0, mo0 + kMaxGroup * kRow, recv, b, g, kPart, kPart,
         (p.mode == kModeDelta) ? mo0 + kMaxGroup * kRow + kMaxGroup * 2 : nullptr);
+    // delta-layers scoring with HEAD_SUM: page scores and the selection, in the stage area
+    if (p.fuse_select) select_tail<WARPS * 32, G>(p, smem, S::kStages, b, g, ex.n, ex.N);
 }
 
 }  // namespace delta

@@ -2,6 +2,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "select_tail.cuh"
 
 namespace delta {
 
@@ -236,6 +237,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     }
     __syncthreads();
     merge_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, recv, b, g, kMaxGroup * D, kMaxGroup * 2);
+    // delta-layers scoring with HEAD_SUM: page scores and the selection, in the stage area
+    if (p.fuse_select) select_tail<kThreads, G>(p, smem, S::kMain, b, g, ex.n, ex.N);
 }
 
 }  // namespace delta

@@ -55,7 +55,8 @@ enum : int { kVarNarrow = 0, kVarWide = 1, kVarShort = 2 };   // tensor-core ker
 constexpr int variant_threads(int v) { return 32 * (v == kVarWide ? kMmaWideWarps : v == kVarShort ? kMmaShortWarps : kWarps); }
 
 struct WsLayout {
-    size_t err, tickets, part_ml, part_o, page_lse, split_ml, logits, total;
+    size_t err, tickets, unit_tickets, seq_tickets, part_ml, part_o, page_lse, split_ml, unit_scores, keys, logits,
+        total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -208,13 +209,18 @@ WsLayout ws_layout(const delta_desc* d, int batch, int max_pages, bool with_logi
     const int S = max_splits_for(d->dtype, d->head_dim, batch, d->num_kv_heads, max_pages);
     const size_t rows = size_t(batch) * d->num_q_heads;
     size_t off = 0;
-    w.err = off;        off += align256(64);
-    w.tickets = off;    off += align256(size_t(batch) * d->num_kv_heads * sizeof(int));
-    w.part_ml = off;    off += align256(rows * S * sizeof(float2));
-    w.part_o = off;     off += align256(rows * S * d->head_dim * sizeof(float));
-    w.page_lse = off;   off += align256(rows * size_t(max_pages) * sizeof(float));
-    w.split_ml = off;   off += align256(rows * S * sizeof(float2));
-    w.logits = off;     off += with_logits ? align256(rows * size_t(max_pages) * kPage * sizeof(float)) : 0;
+    // the counters (error word, tickets) come first: they are the part that must start at zero
+    w.err = off;          off += align256(64);
+    w.tickets = off;      off += align256(size_t(batch) * d->num_kv_heads * sizeof(int));
+    w.unit_tickets = off; off += align256(size_t(batch) * d->num_kv_heads * sizeof(int));
+    w.seq_tickets = off;  off += align256(size_t(batch) * sizeof(int));
+    w.part_ml = off;      off += align256(rows * S * sizeof(float2));
+    w.part_o = off;       off += align256(rows * S * d->head_dim * sizeof(float));
+    w.page_lse = off;     off += align256(rows * size_t(max_pages) * sizeof(float));
+    w.split_ml = off;     off += align256(rows * S * sizeof(float2));
+    w.unit_scores = off;  off += align256(size_t(batch) * d->num_kv_heads * size_t(max_pages) * sizeof(float));
+    w.keys = off;         off += align256(size_t(batch) * size_t(max_pages) * sizeof(uint32_t));
+    w.logits = off;       off += with_logits ? align256(rows * size_t(max_pages) * kPage * sizeof(float)) : 0;
     w.total = off;
     return w;
 }
@@ -595,10 +601,25 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     prm.logits = head_max ? reinterpret_cast<float*>(base + L.logits) : nullptr;
     prm.tickets = reinterpret_cast<int*>(base + L.tickets);
     prm.settled = (mode == kModeSparse && settled) ? 1 : 0;
+    // delta-layers scoring with HEAD_SUM select their pages at the end of the decode kernel
+    prm.fuse_select = (mode == kModeDelta && !head_max) ? 1 : 0;
+    if (prm.fuse_select) {
+        prm.budget_pages = sp->budget_pages;
+        prm.sink_tokens = sp->sink_tokens;
+        prm.recency_tokens = sp->recency_tokens;
+        prm.sel_cnt_out = sel_cnt_out;
+        prm.sel_pages_out = sel_pages_out;
+        prm.sel_stride_out = sel_stride_out;
+        prm.page_scores = page_scores;
+        prm.unit_scores = reinterpret_cast<float*>(base + L.unit_scores);
+        prm.keys = reinterpret_cast<uint32_t*>(base + L.keys);
+        prm.unit_tickets = reinterpret_cast<int*>(base + L.unit_tickets);
+        prm.seq_tickets = reinterpret_cast<int*>(base + L.seq_tickets);
+    }
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     s = launch_decode(d, prm, plan.cluster, plan.variant, pt->batch, st);
-    if (s != DELTA_OK || mode != kModeDelta) return s;
+    if (s != DELTA_OK || mode != kModeDelta || prm.fuse_select) return s;
 
     SelectParams sp2{};
     sp2.indptr = pt->page_indptr;

@@ -23,11 +23,6 @@ struct SelectParams {
     int* err;
 };
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Exclusive block-wide prefix sum of one value per thread (blockDim.x == kSelectThreads).
 __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

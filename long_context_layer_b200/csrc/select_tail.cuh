@@ -1,0 +1,312 @@
+// Page scoring and selection at the end of the delta-layer decode kernel (HEAD_SUM scoring;
+// included by the decode kernels only).
+//
+// DELTA's delta-layers rank the KV pages by the attention they receive and keep the sink pages,
+// the recency window and the best-scoring remaining pages ("DELTA: Dynamic Layer-Aware Token
+// Attention", ai.info summary, "Methodology in Plain English" and "Main Findings" bullet 5).
+// The score of page j is S_j = sum over query heads h of sum over the page's tokens of p[h][t]
+// = sum_h 2^(lse_hj - c_h), with lse_hj the log2-sum-exp of head h's base-2 logits on page j
+// (written by the decode loop) and c_h that head's log2-sum-exp over the whole context.
+//
+// No CTA waits for another.  Every CTA of the grid takes a ticket on its (sequence, KV head)
+// unit once its page terms and split state are visible; the unit's last CTA forms c_h of the
+// unit's G heads from the splits' states and writes the unit's share of every page score; it
+// then takes a ticket on its sequence, and the sequence's last unit sums the KV heads' shares
+// (fixed order: deterministic), finds the k-th largest candidate score by an adaptive-range
+// radix select and writes the ascending selection.
+#pragma once
+
+#include "common.cuh"
+
+namespace delta {
+
+constexpr int kTailList = 128;   // keys the final rank step compares pairwise, at most
+
+// Exclusive prefix sum of one 64-bit value per thread over a block of NTHR threads (a multiple
+// of 32, at most 1024).  `sums` holds NTHR/32 + 1 entries; it is not written again afterwards.
+template <int NTHR>
+__device__ __forceinline__ uint64_t block_scan_u64(uint64_t x, uint64_t* sums, uint64_t& total) {
+    constexpr int W = NTHR / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint64_t w = lane < W ? sums[lane] : 0ull;
+        uint64_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < W) sums[lane] = wi - w;   // exclusive prefix of the warp totals
+        if (lane == 31) sums[W] = wi;        // block total
+    }
+    __syncthreads();
+    total = sums[W];
+    return sums[warp] + incl - x;
+}
+
+// Every thread of the CTA calls this after the output merge.  smem: the kernel's page-stage area,
+// idle by now (free_bytes long, 16-byte aligned).  n, N: the sequence's tokens and pages.
+template <int NTHR, int G>
+__device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char* smem, size_t free_bytes, int b, int g,
+                                         int n, int N) {
+    constexpr int W = NTHR / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, S = p.num_splits, h0 = g * G;
+    const size_t maxp = size_t(p.max_pages);
+
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem);      // [256]
+    uint32_t* list = hist + 256;                              // [kTailList]
+    uint64_t* sums = reinterpret_cast<uint64_t*>(list + kTailList);   // [W + 1]
+    float* s_c = reinterpret_cast<float*>(sums + W + 1);      // [kMaxGroup] per-head normalisers
+    uint32_t* s_u = reinterpret_cast<uint32_t*>(s_c + kMaxGroup);     // [8] flags and broadcasts
+    uint32_t* s_wmin = s_u + 8;                               // [W]
+    uint32_t* s_wmax = s_wmin + W;                            // [W]
+    constexpr size_t kScratch = ((256 + kTailList) * 4 + (W + 1) * 8 + kMaxGroup * 4 + 8 * 4 + 2 * W * 4 + 15) & ~size_t(15);
+    uint32_t* skeys = reinterpret_cast<uint32_t*>(smem + kScratch);
+    const int key_cap = int((free_bytes - kScratch) / 4);
+
+    // 1. this CTA's page terms (page_lse) and split state (split_ml) are visible: arrive at the unit
+    __threadfence();
+    __syncthreads();   // also: no thread still reads the merge records in the stage area
+    if (tid == 0) {
+        const int t = atomicAdd(&p.unit_tickets[b * Hkv + g], 1);
+        const uint32_t last = (t == S - 1) ? 1u : 0u;
+        if (last) p.unit_tickets[b * Hkv + g] = 0;   // ready for the next launch
+        s_u[0] = last;
+    }
+    __syncthreads();
+    if (!s_u[0]) return;
+    __threadfence();
+
+    // 2. c_h of the unit's heads: log2 of the sum of 2^(m) l over the splits' (max, sum) states
+    for (int h = warp; h < G; h += W) {
+        const float2* ps = p.split_ml + (size_t(b) * Hq + h0 + h) * S;
+        float M = -INFINITY, Z = 0.f;
+        for (int base = 0; base < S; base += 32) {
+            const float2 v = (base + lane < S) ? __ldcg(ps + base + lane) : make_float2(-INFINITY, 0.f);
+            float Mr = v.x;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
+            const float Mn = fmaxf(M, Mr);
+            const float mu = (Mn == -INFINITY) ? 0.f : Mn;
+            float z = (v.y > 0.f) ? v.y * exp2_approx(v.x - mu) : 0.f;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            Z = Z * exp2_approx(M - mu) + z;
+            M = Mn;
+        }
+        // no token of the head: every page term is 2^(-inf) = 0
+        if (lane == 0) s_c[h] = (Z > 0.f) ? M + log2_approx(Z) : INFINITY;
+    }
+    __syncthreads();
+
+    // 3. the unit's share of every page score: sum over its G heads of 2^(lse_hj - c_h)
+    {
+        float* us = p.unit_scores + (size_t(b) * Hkv + g) * maxp;
+        const float* pl = p.page_lse + (size_t(b) * Hq + h0) * maxp;
+        for (int j = tid; j < N; j += NTHR) {
+            float v[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) v[h] = __ldcg(pl + size_t(h) * maxp + j);
+            float sc = 0.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h) sc += exp2_approx(v[h] - s_c[h]);
+            us[j] = sc;
+        }
+    }
+
+    // 4. the unit's shares are visible: arrive at the sequence
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int t = atomicAdd(&p.seq_tickets[b], 1);
+        const uint32_t last = (t == Hkv - 1) ? 1u : 0u;
+        if (last) p.seq_tickets[b] = 0;
+        s_u[0] = last;
+    }
+    __syncthreads();
+    if (!s_u[0]) return;
+    __threadfence();
+
+    // 5. page scores (the KV heads' shares summed in head order) and their order keys; the range of
+    //    the candidate keys (pages neither sink nor recency)
+    const int sinkP = min((min(p.sink_tokens, n) + kPage - 1) / kPage, N);
+    const int recStart = (p.recency_tokens > 0) ? min(max(n - p.recency_tokens, 0) / kPage, N) : N;
+    const int k = p.budget_pages;
+    const bool take_all = max(recStart - sinkP, 0) <= k;
+    const bool radix = !take_all && k > 0;
+    uint32_t* keys = (N <= key_cap) ? skeys : p.keys + size_t(b) * maxp;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j = tid; j < N; j += NTHR) {
+        float sc = 0.f;
+        for (int u = 0; u < Hkv; ++u) sc += __ldcg(p.unit_scores + (size_t(b) * Hkv + u) * maxp + j);
+        if (p.page_scores != nullptr) p.page_scores[size_t(b) * maxp + j] = sc;
+        const uint32_t key = order_key(sc);
+        keys[j] = key;
+        if (j >= sinkP && j < recStart) {
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+        }
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+        s_wmin[warp] = kmin;
+        s_wmax[warp] = kmax;
+    }
+    __syncthreads();
+
+    // 6. threshold T and the number of keys equal to T to take (lowest page index first).  Each
+    //    pass buckets the keys of [lo, lo + span] into 256 buckets of width 2^sh, finds the bucket
+    //    holding the kk-th largest and narrows the range to it (span shrinks by 2^8 a pass, so at
+    //    most four passes); once the bucket holds at most kTailList keys they are ranked exactly.
+    uint32_t T = 0, need = 0;
+    if (radix) {
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        for (int w = 0; w < W; ++w) {
+            lo = min(lo, s_wmin[w]);
+            hi = max(hi, s_wmax[w]);
+        }
+        uint32_t span = hi - lo;   // more than k >= 1 candidates: lo <= hi
+        uint32_t kk = uint32_t(k);
+        bool exact = false;
+        for (;;) {
+            const int sh = max(0, 24 - __clz(span));   // (span >> sh) <= 255
+            for (int i = tid; i < 256; i += NTHR) hist[i] = 0u;
+            __syncthreads();
+            for (int j = sinkP + tid; j < recStart; j += NTHR) {
+                const uint32_t key = keys[j];
+                if (key >= lo && key - lo <= span) atomicAdd(&hist[(key - lo) >> sh], 1u);
+            }
+            __syncthreads();
+            if (warp == 0) {   // lane covers buckets 255-8*lane .. 248-8*lane (descending)
+                uint32_t c[8], sum = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    c[i] = hist[255 - 8 * lane - i];
+                    sum += c[i];
+                }
+                uint32_t incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const uint32_t excl = incl - sum;
+                if (excl < kk && kk <= incl) {
+                    uint32_t above = excl;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (above + c[i] >= kk) {
+                            s_u[1] = uint32_t(255 - 8 * lane - i);
+                            s_u[2] = above;
+                            s_u[3] = c[i];
+                            break;
+                        }
+                        above += c[i];
+                    }
+                }
+            }
+            __syncthreads();
+            const uint32_t tb = s_u[1], cnt = s_u[3];
+            kk -= s_u[2];
+            lo += tb << sh;
+            if (sh == 0) {   // the bucket is one key value
+                exact = true;
+                break;
+            }
+            span = min(span - (tb << sh), (1u << sh) - 1u);
+            if (cnt <= uint32_t(kTailList)) break;
+        }
+        if (exact) {
+            T = lo;
+            need = kk;
+        } else {
+            // gather the bucket's keys (at most kTailList) and rank them exactly
+            if (tid == 0) s_u[4] = 0;
+            __syncthreads();
+            for (int base = sinkP; base < recStart; base += NTHR) {   // uniform trip count for the ballot
+                const int j = base + tid;
+                uint32_t key = 0;
+                bool in = false;
+                if (j < recStart) {
+                    key = keys[j];
+                    in = key >= lo && key - lo <= span;
+                }
+                const uint32_t bal = __ballot_sync(0xffffffffu, in);
+                uint32_t slot = 0;
+                if (lane == 0 && bal != 0u) slot = atomicAdd(&s_u[4], uint32_t(__popc(bal)));
+                slot = __shfl_sync(0xffffffffu, slot, 0);
+                if (in) list[slot + __popc(bal & ((1u << lane) - 1u))] = key;
+            }
+            __syncthreads();
+            const int m = int(s_u[4]);
+            // T = the key v with #(> v) < kk <= #(>= v); every holder of v writes the same values
+            for (int i = tid; i < m; i += NTHR) {
+                const uint32_t v = list[i];
+                uint32_t gt = 0, ge = 0;
+                for (int t = 0; t < m; ++t) {
+                    const uint32_t w = list[t];
+                    gt += w > v ? 1u : 0u;
+                    ge += w >= v ? 1u : 0u;
+                }
+                if (gt < kk && kk <= ge) {
+                    s_u[5] = v;
+                    s_u[6] = kk - gt;
+                }
+            }
+            __syncthreads();
+            T = s_u[5];
+            need = s_u[6];
+        }
+    }
+
+    // 7. ascending compaction of sink U recency U {key > T} U {the first `need` keys == T}: each
+    //    thread owns a contiguous run of pages; one scan of the packed (equal, taken) counts gives
+    //    every thread its output position
+    const int per = (N + NTHR - 1) / NTHR;
+    const int jb = min(tid * per, N), je = min(jb + per, N);
+    uint32_t eq_cnt = 0, take_cnt = 0;
+    for (int j = jb; j < je; ++j) {
+        if (take_all || j < sinkP || j >= recStart) {
+            ++take_cnt;
+        } else if (radix) {
+            const uint32_t key = keys[j];
+            if (key > T) ++take_cnt;
+            else if (key == T) ++eq_cnt;
+        }
+    }
+    uint64_t tot;
+    const uint64_t pre = block_scan_u64<NTHR>(uint64_t(eq_cnt) | (uint64_t(take_cnt) << 32), sums, tot);
+    const uint32_t eq_rank = uint32_t(pre), take_rank = uint32_t(pre >> 32);
+    const uint32_t eq_tot = uint32_t(tot), take_tot = uint32_t(tot >> 32);
+    uint32_t pos = take_rank + min(need, eq_rank);
+    uint32_t eq_seen = eq_rank;
+    int32_t* out = p.sel_pages_out + size_t(b) * p.sel_stride_out;
+    for (int j = jb; j < je; ++j) {
+        bool take;
+        if (take_all || j < sinkP || j >= recStart) {
+            take = true;
+        } else if (!radix) {
+            take = false;
+        } else {
+            const uint32_t key = keys[j];
+            take = key > T || (key == T && eq_seen++ < need);
+        }
+        if (take) {
+            if (pos < uint32_t(p.sel_stride_out)) out[pos] = j;
+            ++pos;
+        }
+    }
+    if (tid == 0) p.sel_cnt_out[b] = int(min(take_tot + min(need, eq_tot), uint32_t(p.sel_stride_out)));
+}
+
+}  // namespace delta

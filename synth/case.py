@@ -135,8 +135,8 @@ class Case:
     # ---------------------------------------------------------------- KV values
     def kv_base(self, tensor: int, layer: int, b: int, g: int, pos) -> np.ndarray:
         """Generator values (stored dtype, as float32) with no planting, [len(pos), D]."""
-        return rng.round_to_dtype(
-            rng.normal_block(self.key, tensor, layer, b, g, np.asarray(pos), self.cfg.head_dim), self.cfg.dtype)
+        return rng.normal_block_stored(self.key, tensor, layer, b, g, np.asarray(pos), self.cfg.head_dim,
+                                       self.cfg.dtype)
 
     def kv_logical(self, tensor: int, layer: int, b: int, g: int, n: int | None = None) -> np.ndarray:
         """[n, D] float32 stored K or V of sequence b, kv head g, positions 0..n-1, planting applied."""

@@ -104,6 +104,46 @@ def normal_block(key: int, tensor: int, layer: int, b: int, head: int, pos: np.n
     return normal_from_bits(bits(key, element_counter(tensor, layer, b, head, pos, d)))
 
 
+_HOST_LIB = None
+
+
+def _host_lib():
+    """The C copy of this generator (synth/csrc/synth_host.c), or None when it is not built."""
+    global _HOST_LIB
+    if _HOST_LIB is None:
+        import ctypes
+        import os
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsynth_host.so")
+        if not os.path.exists(path):
+            _HOST_LIB = False
+        else:
+            lib = ctypes.CDLL(path)
+            lib.synth_host_normal_block.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                                    ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
+            lib.synth_host_normal_block.restype = ctypes.c_int
+            _HOST_LIB = lib
+    return _HOST_LIB or None
+
+
+def normal_block_stored(key: int, tensor: int, layer: int, b: int, head: int, pos, dim: int, dtype: str,
+                        use_c: bool = True) -> np.ndarray:
+    """round_to_dtype(normal_block(...), dtype): the stored values, [len(pos), dim] float32.
+
+    Uses the C copy of the generator when it is built (same bits, much faster), else numpy.
+    """
+    lib = _host_lib() if use_c else None
+    if lib is None or dtype not in ("bf16", "f32"):
+        return round_to_dtype(normal_block(key, tensor, layer, b, head, pos, dim), dtype)
+    p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    out = np.empty((p.size, dim), dtype=np.float32)
+    r = lib.synth_host_normal_block(key, tensor, layer, b, head, p.ctypes.data, p.size, dim, float(NORMAL_SCALE),
+                                    1 if dtype == "bf16" else 0, out.ctypes.data)
+    if r != 0:
+        raise ValueError(f"synth_host_normal_block failed ({r})")
+    return out
+
+
 # Salts of the auxiliary draws (host-side choices).  An aux counter is salt << 20 | index.
 SALT_PAGE_PERM = 1
 SALT_CONTEXT = 2

@@ -79,3 +79,18 @@ def test_drift_positions_shift_every_block():
     assert np.array_equal(p0, p1) and np.array_equal(p2, p0 + 256)
     last = case.planted_positions(10, 3, 1, step=999)
     assert last.max() < 16384 - 512
+
+
+def test_host_c_generator_equals_numpy_generator_bit_for_bit():
+    # synth/csrc/synth_host.c restates the generator in C for speed; it must give the same bits
+    assert rng._host_lib() is not None, "libsynth_host.so is not built"
+    r = np.random.default_rng(7)
+    for dtype in ("bf16", "f32"):
+        for _ in range(20):
+            key = int(r.integers(0, 2 ** 63))
+            t, l, b, h = int(r.integers(0, 4)), int(r.integers(0, 64)), int(r.integers(0, 64)), int(r.integers(0, 64))
+            pos = r.integers(0, 1 << 20, size=int(r.integers(1, 50)))
+            dim = int(r.choice([64, 128, 256, 7]))
+            c = rng.normal_block_stored(key, t, l, b, h, pos, dim, dtype)
+            ref = rng.round_to_dtype(rng.normal_block(key, t, l, b, h, pos, dim), dtype)
+            assert np.array_equal(c.view(np.uint32), ref.view(np.uint32))
