@@ -133,9 +133,10 @@ def normal_block_stored(key: int, tensor: int, layer: int, b: int, head: int, po
     Uses the C copy of the generator when it is built (same bits, much faster), else numpy.
     """
     lib = _host_lib() if use_c else None
-    if lib is None or dtype not in ("bf16", "f32"):
-        return round_to_dtype(normal_block(key, tensor, layer, b, head, pos, dim), dtype)
     p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    if lib is None or dtype not in ("bf16", "f32") or (p.size and (p.min() < 0 or p.max() >= MAX_POS)):
+        # (positions outside the counter field keep numpy's wrap-around semantics)
+        return round_to_dtype(normal_block(key, tensor, layer, b, head, p, dim), dtype)
     out = np.empty((p.size, dim), dtype=np.float32)
     r = lib.synth_host_normal_block(key, tensor, layer, b, head, p.ctypes.data, p.size, dim, float(NORMAL_SCALE),
                                     1 if dtype == "bf16" else 0, out.ctypes.data)
