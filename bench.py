@@ -1,18 +1,24 @@
 #!/usr/bin/env python
-"""Benchmark of one DELTA decode step (every layer of the stack) on B200.
+"""Benchmark of the DELTA decode attention stack on B200: one JSON line.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 5]
 
-Default workload: the Qwen-7B-shaped stack in bf16 (28 layers: 0-1 full, delta-layers 2
-and 14, 24 sparse; 28 query / 4 KV heads, head_dim 128; batch 1, context 8192, 16-token
-pages; budget 1024 tokens + 16-token sink + 256-token recency window), synthetic inputs with
-32 planted salient keys per (layer, KV head).  A step is one decode step: kv_append, then
-full, delta or sparse attention, for each of the 28 layers, captured as one CUDA graph.
+Default workload: the largest one that fits one GPU, the drifting decode trajectory
+(drift-48l-b16-16k-bf16): 48 layers (0-1 full, delta-layers 2, 6 and 42, 43 sparse), 40 query /
+8 KV heads, head_dim 128, batch 16, 16385-token start context growing one token per step for
+1000 steps, 16-token pages, budget 2048 tokens + 16-token sink + 512-token recency window, 32
+planted salient keys per (layer, sequence, KV head) that move by 256 tokens every 100 steps
+(about 52 GB of KV cache).  A step is one decode step: the kv_append of every layer, then full,
+delta or sparse attention for each of the 48 layers, replayed as one CUDA graph.
 
-Timing: W untimed replays, then K timed replays, L2 flushed (a 2x L2-sized write) before every
-replay outside the events; CUDA events on the replay stream; max over ranks.  Prints one JSON
-line.  With --gpus N > 1 (torchrun) every rank runs an independent replica (the path does
-not shard across GPUs) and the reported time is the slowest rank's.
+Timing: every step of the trajectory runs; K of them (all by default), evenly spread, are timed
+with CUDA events on the replay stream, L2 flushed before each timed replay (outside the
+events); W untimed replays of the first step come first.  The value is the mean time of a timed
+step (with --gpus N, N independent replicas: the slowest replica's mean).  The same line carries
+the kernel rooflines, the same build's all-full stack, the attended-token reduction, an
+end-to-end time through the public API with host buffers, the fp64 oracle timed on the host
+cores, and (on rank 0) the oracle's verdict on every delta-layer selection of every sequence at
+the sampled steps.  --config 1..4 time one decode step of the other workloads instead.
 """
 from __future__ import annotations
 
@@ -30,24 +36,30 @@ sys.path.insert(0, ROOT)
 
 METRIC = "us_per_decode_step_layer_stack"
 UNIT = "us/step"
+L2_NOTE = "flushed before every timed replay (2xL2 write, then 2xL2 read), outside the events"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (trajectory default: every step; single-step workloads: 200)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
+    ap.add_argument("--checks", type=int, default=-1,
+                    help="trajectory steps whose delta-layer selections (every sequence) the oracle checks: "
+                         "-1 every step at a drift boundary (0, 99, 100, ..., last), 0 none, m the first m of those")
+    ap.add_argument("--oracle-procs", type=int, default=0, help="oracle worker processes (0: every host core)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the summaries of the 64k and 8k workloads")
     ap.add_argument("--print-source-hash", action="store_true", help="print the kernel-source hash and exit")
-    ap.add_argument("--drift-checks", type=int, default=10, help="oracle selection checks along a trajectory")
     ap.add_argument("--reduce", choices=["sum", "max"], default="sum",
                     help="head aggregation of the page score: sum (default) or the page's max rule")
     ap.add_argument("--delta-sweep", type=str, default="",
                     help="comma list of delta-layer counts: time the step for each (spread placement)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -64,25 +76,27 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str, kind: str = "full_layer"):
-    """DRAM bytes per launch of the decode kernel in a full or sparse layer, from the committed ncu
-    summary of this workload, or None when the kernels changed since that capture."""
-    path = os.path.join(ROOT, "profiles", f"decode_{kind}_{workload}.md")
+def profiled_traffic(workload: str, kind: str):
+    """(DRAM bytes per launch, summary file) of the decode kernel of a full, delta or sparse layer
+    from the committed ncu summary of this workload, or (None, why) when there is none or the
+    kernels changed since that capture."""
+    name = f"decode_{kind}_{workload}.md"
+    path = os.path.join(ROOT, "profiles", name)
     try:
         text = open(path).read()
     except OSError:
-        return None
+        return None, "no ncu summary for this workload"
     fields = {}
     for line in text.splitlines():
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             fields[k.strip()] = v.strip().strip("`")
     if fields.get("kernel_sources_sha256") != kernel_source_hash():
-        return None
+        return None, f"profiles/{name} was taken on other kernel sources"
     try:
-        return int(fields["traffic_bytes_per_launch"])
+        return int(fields["traffic_bytes_per_launch"]), f"profiles/{name}"
     except (KeyError, ValueError):
-        return None
+        return None, f"profiles/{name} has no traffic figure"
 
 
 def load_peaks():
@@ -146,6 +160,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
+def gpu_index(device) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[device.index])
+        except (ValueError, IndexError):
+            return device.index
+    return device.index
+
+
 def dist_init():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
@@ -177,9 +201,28 @@ def barrier(dist, device):
         torch.cuda.synchronize(device)
 
 
+def config_dict(cfg, reduce: str = "sum", world: int = 1) -> dict:
+    """The workload, as both arms of the benchmark report it."""
+    d = {"workload": cfg.name, "layers": cfg.num_layers, "delta_layers": list(cfg.delta_layers),
+         "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim, "batch": cfg.batch,
+         "page_size": cfg.page_size, "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
+         "recency_tokens": cfg.recency_tokens, "score": f"head {reduce}", "parallelism": f"replicas x{world}",
+         "l2": L2_NOTE}
+    if cfg.context_list:
+        d["context"] = list(cfg.context_list)
+    elif cfg.context:
+        d["context"] = cfg.context
+    else:
+        d["context_range"] = list(cfg.context_range)
+    if cfg.steps > 1:
+        d.update({"trajectory_steps": cfg.steps, "drift_every": cfg.drift_every, "drift_shift": cfg.drift_shift})
+    return d
+
+
 # ---------------------------------------------------------------------------- accounting
 def attended_tokens(cfg, case):
-    """(delta_stack_tokens, full_stack_tokens) attended per step, summed over layers and sequences.
+    """(delta_stack_tokens, full_stack_tokens, full_tokens_per_layer, sparse_tokens_per_layer) attended per
+    step, summed over layers and sequences.
 
     Sparse layers attend the tokens of the selected pages: every sink/recency page plus k
     candidate pages, the last page partial (computed from the selection rule's page counts).
@@ -203,10 +246,19 @@ def attended_tokens(cfg, case):
     return n_dense * full_tok + n_sparse * sparse_tok, len(kinds) * full_tok, full_tok, sparse_tok
 
 
-# ---------------------------------------------------------------------------- reference arm
+def delta_page_term_bytes(cfg, case) -> int:
+    """Bytes a delta-layer moves for its page scores beyond attention: each (head, page) log-sum-exp
+    and each (KV head, page) score share, written once and read once, plus the selection."""
+    pages = sum(-(-int(n) // cfg.page_size) for n in case.n.tolist())
+    sel = cfg.batch * (cfg.budget_pages + 40) * 4
+    return pages * (cfg.num_q_heads + cfg.num_kv_heads) * 4 * 2 + sel
+
+
+# ---------------------------------------------------------------------------- the oracle leg
 class OracleSample:
-    """The fp64 oracle on one full, one delta and one sparse layer of sequence 0 (inputs
-    generated once, outside any timing); a step estimate scales them to the whole stack."""
+    """The fp64 oracle (test infrastructure: only this leg of the benchmark runs it) on one full,
+    one delta and one sparse layer of sequence 0, inputs generated once outside any timing; a
+    step estimate scales them to the whole stack and batch."""
 
     def __init__(self, cfg, case):
         import numpy as np
@@ -235,20 +287,22 @@ class OracleSample:
         return O.select_pages(O.page_scores(p, c.page_size), self.n, c.page_size, c.budget_pages, c.sink_tokens,
                               c.recency_tokens)
 
-    def layer_us(self, min_seconds: float = 0.0, max_reps: int = 200) -> dict:
-        """Wall-clock microseconds per layer of each kind for one sequence."""
+    def layer_us(self, min_seconds: float) -> dict:
+        """Wall-clock microseconds per layer of each kind for one sequence (each kind repeated for
+        about a third of min_seconds, at least twice, the first call not timed)."""
         O, c = self.O, self.cfg
         fns = {"full": lambda: O.full_attention(*self.data[self.l_full]),
                "delta": lambda: self._select(self.data[self.l_delta]),
                "sparse": lambda: O.sparse_attention(*self.data[self.l_sparse], self.sel, c.page_size)}
         out = {}
         for name, fn in fns.items():
+            fn()
             k, t0 = 0, time.perf_counter()
             while True:
                 fn()
                 k += 1
                 el = time.perf_counter() - t0
-                if el >= min_seconds / 3 or k >= max_reps:
+                if k >= 2 and el >= min_seconds / 3:
                     break
             out[name] = el / k * 1e6
         return out
@@ -260,6 +314,12 @@ class OracleSample:
         full_us = self.cfg.batch * len(self.kinds) * times["full"]
         return delta_us, full_us
 
+    def describe(self, times: dict, seconds: float) -> str:
+        c = self.cfg
+        return (f"fp64 numpy oracle on the host cores, sequence 0 of {c.name}: one full / delta / sparse layer, each "
+                f"repeated for ~{seconds / 3:.1f} s ({', '.join(f'{k} {v:.0f} us' for k, v in times.items())}), "
+                f"scaled to the {c.num_layers}-layer step x batch {c.batch}")
+
 
 def blas_threads():
     try:
@@ -270,7 +330,17 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def cpu_baseline_leg(cfg, case, seconds: float) -> dict:
+    sample = OracleSample(cfg, case)
+    times = sample.layer_us(min_seconds=seconds)
+    d_us, f_us = sample.step_us(times)
+    return {"value": round(d_us, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": sample.describe(times, seconds), "full_stack_value": round(f_us, 1)}
+
+
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, timed on the host cores on a bounded sample of
+    each step (rank 0 only)."""
     dist, rank, world, local = dist_init()
     if rank != 0:
         if dist is not None:
@@ -281,25 +351,23 @@ def run_reference(args):
     cfg = C.CONFIGS[args.config]
     case = Case(cfg)
     sample = OracleSample(cfg, case)
-    per_step = []
-    desc = None
-    for i in range(args.warmup + args.steps):
-        times = sample.layer_us(max_reps=1)
+    K = args.steps if args.steps else 20
+    per_step_s = max(0.3, min(args.cpu_seconds / max(K + args.warmup, 1), 3.0))
+    per_step, desc = [], None
+    for i in range(args.warmup + K):
+        times = sample.layer_us(min_seconds=per_step_s)
         d_us, _ = sample.step_us(times)
         if i >= args.warmup:
             per_step.append(d_us)
         desc = times
     value = statistics.mean(per_step)
-    cores = blas_threads()
-    sample = (f"fp64 numpy oracle, sequence 0, one full / delta / sparse layer per step "
-              f"({', '.join(f'{k} {v:.0f} us' for k, v in desc.items())}), scaled to {cfg.num_layers} layers "
-              f"x batch {cfg.batch}")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1000, 6),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "batch": cfg.batch, "context": int(case.n.max()), "layers": cfg.num_layers},
-        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(value / 1000, 6), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, args.reduce, world),
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample.describe(desc, per_step_s)},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -307,308 +375,411 @@ def run_reference(args):
         dist.destroy_process_group()
 
 
-# ---------------------------------------------------------------------------- drifting trajectory
-def run_trajectory(args, cfg):
-    """The drifting workload: one CUDA graph per decode step replayed along the trajectory, the
-    cache growing one token per step and the planted keys moving every `drift_every` steps.
-    Reports per-step latency and, on sampled steps, the rate at which the GPU selection of
-    sequence 0 at the first delta-layer matches the fp64 oracle's."""
-    import numpy as np
-    import torch
-    from long_context_layer_b200.stack import DeltaStack
-    from synth.trajectory import Trajectory
+# ---------------------------------------------------------------------------- GPU measurement
+class Gpu:
+    """L2 flush buffers and event timing on the current stream of one device."""
 
-    dist, rank, world, local = dist_init()
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    tr = Trajectory(cfg, device=device)
-    dc = tr.dc
-    stack = DeltaStack(cfg.layer_kinds(), cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr,
-                       dc.indices, dc.kv_len, tr.case0.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages,
-                       cfg.sink_tokens, cfg.recency_tokens)
-    tr.prepare(0)
-    g = stack.capture(dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
-    flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
-    steps = min(args.steps, cfg.steps)
-    check_every = max(steps // max(args.drift_checks, 1), 1)
-    checks = set(range(0, steps, check_every)) if args.drift_checks > 0 else set()
-    lat, matched, checked = [], 0, 0
-    ld = cfg.layer_kinds().index("delta")
-    for step in range(steps):
-        tr.prepare(step)
-        for _ in range(args.warmup if step == 0 else 0):
-            g.replay()
-        flush.fill_(1)
-        flush_rd.sum()
-        barrier(dist, device)
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        g.replay()
-        s1.record(stream)
-        s1.synchronize()
-        lat.append(s0.elapsed_time(s1) * 1000.0)
-        if rank == 0 and step in checks:
-            from oracle import delta_oracle as O
-            from synth import rng
-            case = tr.case_at(step)
-            n = int(case.n[0])
-            K = np.stack([case.kv_logical(rng.T_K, ld, 0, h) for h in range(cfg.num_kv_heads)]).astype(np.float64)
-            V = np.stack([case.kv_logical(rng.T_V, ld, 0, h) for h in range(cfg.num_kv_heads)]).astype(np.float64)
-            _, p = O.full_attention(case.q(ld)[0].astype(np.float64), K, V)
-            ref = O.select_pages(O.page_scores(p, cfg.page_size), n, cfg.page_size, cfg.budget_pages,
-                                 cfg.sink_tokens, cfg.recency_tokens)
-            matched += int(stack.selection(stack.delta_layers.index(ld))[0] == ref)
-            checked += 1
-    per = np.array(lat)
-    us = max_over_ranks(dist, float(per.mean()), device)
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(us, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": round(us / 1000, 6), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": cfg.name, "layers": cfg.num_layers, "delta_layers": list(cfg.delta_layers),
-                       "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
-                       "batch": cfg.batch, "start_context": int(tr.case0.n.max()), "drift_every": cfg.drift_every,
-                       "drift_shift": cfg.drift_shift, "budget_tokens": cfg.budget_tokens,
-                       "l2": "flushed before every timed replay (2xL2 write, then 2xL2 read)"},
-            "trajectory": {"per_step_us": {"mean": round(float(per.mean()), 3),
-                                           "median": round(float(np.median(per)), 3),
-                                           "p99": round(float(np.percentile(per, 99)), 3),
-                                           "first": round(float(per[0]), 3), "last": round(float(per[-1]), 3)},
-                           "selection_match_rate": (round(matched / checked, 4) if checked else None),
-                           "selection_checks": checked,
-                           "selection_check": "sequence 0, first delta-layer, exact match with the fp64 oracle"},
-            "gpu_launches": stack.launches_per_step() * steps,
-        }
-        print(json.dumps(line), flush=True)
-    del g
-    stack.graph = None
-    if dist is not None:
-        dist.destroy_process_group()
+    def __init__(self, device, dist=None):
+        import torch
+        self.torch = torch
+        self.device, self.dist = device, dist
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        self.flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
+        self.flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+        self.stream = torch.cuda.current_stream(device)
 
+    def flush_l2(self):
+        # write a buffer twice the size of L2, then read another one, so no dirty lines of the flush
+        # are left to be written back inside the timed region
+        self.flush.fill_(1)
+        self.flush_rd.sum()
 
-# ---------------------------------------------------------------------------- our arm
-def run_ours(args):
-    import torch
-    from long_context_layer_b200 import _native as NAT
-    from long_context_layer_b200.stack import DeltaStack
-    from synth import configs as C
-    from synth.case import Case
-    from synth.gpu import DeviceCase
-
-    dist, rank, world, local = dist_init()
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    cfg = C.CONFIGS[args.config]
-    case = Case(cfg)
-    dc = DeviceCase(case, device=device, prefill="append")
-    kinds = cfg.layer_kinds()
-    reduce = NAT.DELTA_HEAD_MAX if args.reduce == "max" else NAT.DELTA_HEAD_SUM
-    mk = lambda kk: DeltaStack(kk, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr, dc.indices,
-                               dc.kv_len, case.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages,
-                               cfg.sink_tokens, cfg.recency_tokens, reduce=reduce)
-    delta_stack = mk(kinds)
-    full_stack = mk(["full"] * cfg.num_layers)
-    args_step = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
-    g_delta = delta_stack.capture(*args_step)
-    g_full = full_stack.capture(*args_step)
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
-    flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
-
-    def flush_l2():
-        # write a buffer twice the size of L2, then read another one, so no dirty lines of the
-        # flush are left to be written back inside the timed region
-        flush.fill_(1)
-        flush_rd.sum()
-
-    def timed(replay, k, warm):
+    def timed(self, replay, k: int, warm: int) -> list:
+        torch = self.torch
         for _ in range(warm):
-            flush_l2()
+            self.flush_l2()
             replay()
-        barrier(dist, device)
+        barrier(self.dist, self.device)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
         for s, e in ev:
-            flush_l2()
-            s.record(stream)
+            self.flush_l2()
+            s.record(self.stream)
             replay()
-            e.record(stream)
-        barrier(dist, device)
+            e.record(self.stream)
+        barrier(self.dist, self.device)
         return [s.elapsed_time(e) * 1000.0 for s, e in ev]   # us
 
-    sampler = ClockSampler(device.index if not os.environ.get("CUDA_VISIBLE_DEVICES") else
-                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[device.index]))
-    sampler.start()
-    time.sleep(0.3)
-    t_delta = timed(g_delta.replay, args.steps, args.warmup)
-    clocks = sampler.stop()
-    t_full = timed(g_full.replay, max(args.steps // 2, 3), 3)
-    us_delta = max_over_ranks(dist, statistics.mean(t_delta), device)
-    us_full = max_over_ranks(dist, statistics.mean(t_full), device)
+    def mean_us(self, replay, k: int, warm: int = 3) -> float:
+        return max_over_ranks(self.dist, statistics.mean(self.timed(replay, k, warm)), self.device)
 
-    # -- dominant kernel: the decode kernel of a full layer, timed alone (one launch per call)
-    st = stream.cuda_stream
-    d0 = delta_stack
-    layer0 = 0
 
-    def full_call():
-        NAT.full_attn(d0.desc, d0.pt, dc.q[layer0], dc.k_pools[layer0], dc.v_pools[layer0], dc.out[layer0],
-                      d0.workspace, d0.ws_bytes, st)
+def make_stacks(cfg, case, dc, reduce):
+    from long_context_layer_b200 import _native as NAT
+    from long_context_layer_b200.stack import DeltaStack
+    red = NAT.DELTA_HEAD_MAX if reduce == "max" else NAT.DELTA_HEAD_SUM
+    mk = lambda kk: DeltaStack(kk, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr, dc.indices,
+                               dc.kv_len, case.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages,
+                               cfg.sink_tokens, cfg.recency_tokens, reduce=red)
+    return mk
 
-    t_kernel = timed(full_call, max(args.steps, 20), 3)
-    us_kernel = max_over_ranks(dist, statistics.mean(t_kernel), device)
 
-    # -- per-call breakdown (each call timed alone, L2 flushed before it)
+def kernel_measurements(gpu, cfg, case, dc, d0, us_full_stack: float, k: int, with_breakdown: bool = True) -> dict:
+    """Rooflines of the three decode kernels of a step and a per-call breakdown.
+
+    Each kernel runs L times in one CUDA graph (the layers' own q and pools), timed like the steps;
+    the per-launch average is its steady-state duration.  Sparse layers run on the first
+    delta-layer's selection, all but the first launch through the settled entry, as in a step;
+    the full-layer figure comes from the all-full stack graph (L launches + 1 append, the append
+    charged to the kernel).  Algorithmic bytes: the attended tokens' K and V of every sequence,
+    plus q and o (delta-layers also their page-score terms).
+    """
+    import torch
+    from long_context_layer_b200 import _native as NAT
+    st = gpu.stream.cuda_stream
+    kinds = cfg.layer_kinds()
+    L = cfg.num_layers
     lk = kinds.index("delta")
     ls = kinds.index("sparse")
     di = d0.delta_layers.index(lk)
+    e = 2 if cfg.dtype == "bf16" else 4
+    kvtok = 2 * cfg.num_kv_heads * cfg.head_dim * e
+    qo = 2 * cfg.batch * cfg.num_q_heads * cfg.head_dim * e
+    _, _, full_tok, sparse_tok = attended_tokens(cfg, case)
+    peak, peak_kind = load_peaks()
 
-    def append_call():
-        NAT.kv_append(d0.desc, d0.pt, dc.k_new[0], dc.v_new[0], dc.k_pools[0], dc.v_pools[0], st)
+    def graph_of(calls):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(gpu.device)
+        side.wait_stream(gpu.stream)
+        with torch.cuda.stream(side):
+            calls(side.cuda_stream)   # warm outside capture (per-device kernel attributes)
+        gpu.stream.wait_stream(side)
+        with torch.cuda.graph(g):
+            calls(torch.cuda.current_stream(gpu.device).cuda_stream)
+        return g
 
-    def select_call():
-        NAT.select_attn(d0.desc, d0.pt, d0.sp, dc.q[lk], dc.k_pools[lk], dc.v_pools[lk], dc.out[lk], d0.sel_cnt[di],
-                        d0.sel_pages[di], d0.sel_stride, None, d0.workspace, d0.ws_bytes, st)
-
-    def sparse_call():
-        NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[ls], dc.k_pools[ls],
-                        dc.v_pools[ls], dc.out[ls], d0.workspace, d0.ws_bytes, st)
-
-    # -- the sparse-layer decode (24 of the 28 launches of a step): L launches of it in one graph,
-    #    all on the delta-layer's selection, timed like the steps; per-launch average.  As in the
-    #    step, every launch after the first uses the settled entry (its predecessor is sparse).
-    lay = list(range(cfg.num_layers))
-    sg = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(device)
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        for l in lay:   # warm outside capture (per-device kernel attributes)
-            NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[l], dc.k_pools[l],
-                            dc.v_pools[l], dc.out[l], d0.workspace, d0.ws_bytes, side.cuda_stream)
-    stream.wait_stream(side)
-    with torch.cuda.graph(sg):
-        cs = torch.cuda.current_stream(device).cuda_stream
-        for l in lay:
+    def sparse_calls(s):
+        for l in range(L):
             fn = NAT.sparse_attn if l == 0 else NAT.sparse_attn_settled
             fn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[l], dc.k_pools[l],
-               dc.v_pools[l], dc.out[l], d0.workspace, d0.ws_bytes, cs)
-    t_sparse = timed(sg.replay, max(args.steps // 2, 10), 3)
-    us_sparse_launch = max_over_ranks(dist, statistics.mean(t_sparse), device) / len(lay)
-    del sg
+               dc.v_pools[l], dc.out[l], d0.workspace, d0.ws_bytes, s)
 
-    n_b = max(args.steps // 2, 10)
-    breakdown = {name: round(max_over_ranks(dist, statistics.mean(timed(fn, n_b, 3)), device), 3)
-                 for name, fn in (("kv_append", append_call), ("full_attn", full_call),
-                                  ("select_attn", select_call), ("sparse_attn", sparse_call))}
-    e = 2 if cfg.dtype == "bf16" else 4
-    kv_bytes = int(case.n.sum()) * 2 * cfg.num_kv_heads * cfg.head_dim * e
-    qo_bytes = 2 * cfg.batch * cfg.num_q_heads * cfg.head_dim * e
-    alg_bytes = kv_bytes + qo_bytes
-    peak, peak_kind = load_peaks()
-    # The full-attention stack is one graph of L launches of this same decode kernel (plus one
-    # append launch), timed with CUDA events: its per-launch average is the kernel's duration in
-    # steady state (the append is charged to it, which only lowers the figure).  The single call
-    # timed above also carries a launch latency no graph pays; it is reported alongside.
-    us_launch = us_full / cfg.num_layers
-    achieved = alg_bytes / (us_launch * 1e-6) / 1e9
-    achieved_single = alg_bytes / (us_kernel * 1e-6) / 1e9
-    # sparse layers: the tokens of the selected pages of every sequence
-    _, _, _, sparse_tok = attended_tokens(cfg, case)
-    alg_sparse = sparse_tok * 2 * cfg.num_kv_heads * cfg.head_dim * e + qo_bytes
-    achieved_sparse = alg_sparse / (us_sparse_launch * 1e-6) / 1e9
+    def delta_calls(s):
+        for l in range(L):
+            NAT.select_attn(d0.desc, d0.pt, d0.sp, dc.q[l], dc.k_pools[l], dc.v_pools[l], dc.out[l], d0.sel_cnt[di],
+                            d0.sel_pages[di], d0.sel_stride, None, d0.workspace, d0.ws_bytes, s)
+        # leave the first delta-layer's own selection in place for the sparse launches
+        NAT.select_attn(d0.desc, d0.pt, d0.sp, dc.q[lk], dc.k_pools[lk], dc.v_pools[lk], dc.out[lk], d0.sel_cnt[di],
+                        d0.sel_pages[di], d0.sel_stride, None, d0.workspace, d0.ws_bytes, s)
+
+    g_delta = graph_of(delta_calls)
+    us_delta_launch = gpu.mean_us(g_delta.replay, k) / (L + 1)
+    g_sparse = graph_of(sparse_calls)
+    us_sparse_launch = gpu.mean_us(g_sparse.replay, k) / L
+    del g_delta, g_sparse
+
+    def roof(kernel, alg, us, launches, timing, kind):
+        traffic, source = profiled_traffic(cfg.name, kind)
+        achieved = alg / (us * 1e-6) / 1e9
+        return {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": peak_kind, "alg_bytes_per_launch": int(alg),
+                "us_per_launch": round(us, 3), "launches_per_step": launches, "timing": timing,
+                "traffic": traffic, "traffic_source": source}
+
     n_sparse = kinds.count("sparse")
+    n_delta = kinds.count("delta")
+    out = {
+        "roofline": roof("decode_mma_kernel, sparse layer (selected pages, split-KV, cluster merge)",
+                         sparse_tok * kvtok + qo, us_sparse_launch, n_sparse,
+                         "graph of L sparse launches on a delta-layer's selection (all but the first through the "
+                         "settled entry, as in the step) / L, CUDA events, L2 flushed", "sparse_layer"),
+        "roofline_full_layer": roof("decode_mma_kernel, full layer (split-KV, cluster merge)",
+                                    full_tok * kvtok + qo, us_full_stack / L, L - n_sparse - n_delta,
+                                    "all-full stack graph (L launches + 1 append) / L, CUDA events, L2 flushed",
+                                    "full_layer"),
+        "roofline_delta_layer": roof("decode_mma_kernel, delta layer (full attention + page scores + selection in "
+                                     "the last CTA of each sequence)",
+                                     full_tok * kvtok + qo + delta_page_term_bytes(cfg, case), us_delta_launch,
+                                     n_delta, "graph of L + 1 delta-layer launches / (L + 1), CUDA events, L2 flushed",
+                                     "delta_layer"),
+    }
+    if cfg.dtype != "bf16":
+        for key in out:
+            out[key]["kernel"] = out[key]["kernel"].replace("decode_mma_kernel", "decode_kernel (fp32)")
+    if with_breakdown:
+        def append_call():
+            NAT.kv_append(d0.desc, d0.pt, dc.k_new[0], dc.v_new[0], dc.k_pools[0], dc.v_pools[0], st)
 
-    # -- end to end through the public API: every step the step's inputs (q, k_new, v_new) come
-    #    from one pinned host staging buffer in one copy, the step runs (the same calls, captured in
-    #    a graph over views of the device staging buffer) and every layer's output goes back to
-    #    pinned host memory
+        def full_call():
+            NAT.full_attn(d0.desc, d0.pt, dc.q[0], dc.k_pools[0], dc.v_pools[0], dc.out[0], d0.workspace,
+                          d0.ws_bytes, st)
+
+        def select_call():
+            NAT.select_attn(d0.desc, d0.pt, d0.sp, dc.q[lk], dc.k_pools[lk], dc.v_pools[lk], dc.out[lk],
+                            d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, None, d0.workspace, d0.ws_bytes, st)
+
+        def sparse_call():
+            NAT.sparse_attn(d0.desc, d0.pt, d0.sel_cnt[di], d0.sel_pages[di], d0.sel_stride, dc.q[ls],
+                            dc.k_pools[ls], dc.v_pools[ls], dc.out[ls], d0.workspace, d0.ws_bytes, st)
+
+        out["breakdown_us_per_call"] = {
+            name: round(gpu.mean_us(fn, k), 3)
+            for name, fn in (("kv_append", append_call), ("full_attn", full_call), ("select_attn", select_call),
+                             ("sparse_attn", sparse_call))}
+        out["breakdown_note"] = "each call launched alone from the host, L2 flushed before it (includes launch latency)"
+    out["roofline"]["share_of_step"] = None
+    return out
+
+
+def e2e_measure(gpu, cfg, dc, mk, k: int) -> dict:
+    """End to end through the public API with host buffers: every step the step's inputs (q, k_new,
+    v_new) go from one pinned host staging buffer to the device in one copy, the step runs (the
+    same C-ABI calls, captured in a graph over views of the device staging buffer) and every
+    layer's output comes back to pinned host memory."""
+    import torch
     nq, nk = dc.q.numel(), dc.k_new.numel()
     in_h = torch.cat([dc.q.reshape(-1), dc.k_new.reshape(-1), dc.v_new.reshape(-1)]).cpu().pin_memory()
-    in_d = torch.empty_like(in_h, device=device)
+    in_d = torch.empty_like(in_h, device=gpu.device)
     in_d.copy_(in_h)
     q_v = in_d[:nq].view_as(dc.q)
     kn_v = in_d[nq:nq + nk].view_as(dc.k_new)
     vn_v = in_d[nq + nk:].view_as(dc.v_new)
     out_h = torch.empty_like(dc.out, device="cpu").pin_memory()
-    e2e_stack = mk(kinds)
-    g_e2e = e2e_stack.capture(q_v, kn_v, vn_v, dc.k_pools, dc.v_pools, dc.out)
+    stack = mk(cfg.layer_kinds())
+    g = stack.capture(q_v, kn_v, vn_v, dc.k_pools, dc.v_pools, dc.out)
 
-    def e2e_step():
+    def step():
         in_d.copy_(in_h, non_blocking=True)
-        g_e2e.replay()
+        g.replay()
         out_h.copy_(dc.out, non_blocking=True)
 
-    t_e2e = timed(e2e_step, args.steps, 3)
-    us_e2e = max_over_ranks(dist, statistics.mean(t_e2e), device)
-    h2d = in_h.numel() * e
-    d2h = out_h.numel() * e
-    del g_e2e
-    e2e_stack.graph = None
+    us = gpu.mean_us(step, k)
+    e = in_h.element_size()
+    del g
+    stack.graph = None
+    return {"value": round(us, 3), "unit": UNIT, "h2d_bytes_per_step": in_h.numel() * e,
+            "d2h_bytes_per_step": out_h.numel() * e,
+            "how": "pinned host inputs -> device (one copy), graph replay of the step's C-ABI calls, every "
+                   "layer's output -> pinned host; CUDA events around the three"}
 
+
+def run_static(args, cfg, dist, rank, world, device, headline: bool = True) -> dict:
+    """One decode step of a single-step workload: the DELTA stack, the all-full stack, the kernel
+    rooflines, a per-call breakdown, e2e and the oracle on the host cores."""
+    import torch
+    from synth.case import Case
+    from synth.gpu import DeviceCase
+    case = Case(cfg)
+    dc = DeviceCase(case, device=device, prefill="append")
+    mk = make_stacks(cfg, case, dc, args.reduce)
+    delta_stack = mk(cfg.layer_kinds())
+    full_stack = mk(["full"] * cfg.num_layers)
+    step_args = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    g_delta = delta_stack.capture(*step_args)
+    g_full = full_stack.capture(*step_args)
+    gpu = Gpu(device, dist)
+    K = args.steps if args.steps else 200
+    k2 = max(min(K, 100), 10)
+    sampler = ClockSampler(gpu_index(device))
+    sampler.start()
+    time.sleep(0.3)
+    t_delta = gpu.timed(g_delta.replay, K, args.warmup)
+    clocks = sampler.stop()
+    us_delta = max_over_ranks(dist, statistics.mean(t_delta), device)
+    us_full = gpu.mean_us(g_full.replay, k2)
+    km = kernel_measurements(gpu, cfg, case, dc, delta_stack, us_full, k2, with_breakdown=headline)
+    n_sparse = cfg.layer_kinds().count("sparse")
+    km["roofline"]["share_of_step"] = round(n_sparse * km["roofline"]["us_per_launch"] / us_delta, 3)
     tok_delta, tok_full, _, _ = attended_tokens(cfg, case)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = OracleSample(cfg, case)
-        times = sample.layer_us(min_seconds=args.cpu_seconds)
-        d_us, f_us = sample.step_us(times)
-        cpu = {"value": round(d_us, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": ("fp64 numpy oracle on the host cores, sequence 0, one full / delta / sparse layer "
-                          f"repeated for ~{args.cpu_seconds:.0f} s ({', '.join(f'{k} {v:.0f} us' for k, v in times.items())}), "
-                          f"scaled to the {cfg.num_layers}-layer step x batch {cfg.batch}"),
-               "full_stack_value": round(f_us, 1)}
-    launches = delta_stack.launches_per_step() * args.steps
-    if rank == 0:
-        line = {
-            # whole job: N replicas each finish a decode step in us_delta (slowest rank), so the job
-            # spends us_delta / N per decode step; ms_per_step is one step iteration of the job
-            "metric": METRIC, "value": round(us_delta / world, 3), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us_delta / 1000, 6),
-            "replica_step_us": round(us_delta, 3), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": cfg.name, "layers": cfg.num_layers, "delta_layers": list(cfg.delta_layers),
-                       "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
-                       "batch": cfg.batch, "context": int(case.n.max()), "page_size": cfg.page_size,
-                       "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
-                       "recency_tokens": cfg.recency_tokens, "l2": "flushed before every timed replay (2xL2 write, then 2xL2 read)",
-                       "parallelism": f"replicas x{world}", "score": f"head {args.reduce}"},
-            "full_stack_us": round(us_full, 3),
-            "speedup_vs_full_stack": round(us_full / us_delta, 3),
-            "attended_token_reduction": round(tok_full / tok_delta, 3),
-            # the kernel that dominates the step: the decode kernel of the sparse layers
-            "roofline": {"kernel": "decode_mma_kernel, sparse layer (selected pages, split-KV, cluster merge)",
-                         "bound": "hbm", "achieved": round(achieved_sparse, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved_sparse / peak, 4), "peak_source": peak_kind,
-                         "alg_bytes_per_launch": alg_sparse, "us_per_launch": round(us_sparse_launch, 3),
-                         "launches_per_step": n_sparse,
-                         "share_of_step": round(n_sparse * us_sparse_launch / us_delta, 3),
-                         "timing": ("graph of L sparse launches on the delta-layer's selection (all but the first "
-                                    "through the settled entry, as in the step) / L, CUDA events, L2 flushed"),
-                         "traffic": profiled_traffic(cfg.name, "sparse_layer")},
-            "roofline_full_layer": {"kernel": "decode_mma_kernel, full layer (split-KV, cluster merge)", "bound": "hbm",
-                                    "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                                    "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                                    "alg_bytes_per_launch": alg_bytes, "us_per_launch": round(us_launch, 3),
-                                    "launches_per_step": len(kinds) - n_sparse,
-                                    "timing": "full-attention stack graph (L launches + 1 append) / L, CUDA events, L2 flushed",
-                                    "single_call_us": round(us_kernel, 3),
-                                    "single_call_frac": round(achieved_single / peak, 4),
-                                    "traffic": profiled_traffic(cfg.name, "full_layer")},
-            "breakdown_us_per_call": breakdown,
-            "e2e": {"value": round(us_e2e / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line), flush=True)
-    # release graphs before tearing down the process group
+    res = {"us_per_step": round(us_delta, 3), "full_stack_us": round(us_full, 3),
+           "speedup_vs_full_stack": round(us_full / us_delta, 3),
+           "attended_token_reduction": round(tok_full / tok_delta, 3)}
+    res.update(km)
+    if headline:
+        res["e2e"] = e2e_measure(gpu, cfg, dc, mk, K)
+        res["clocks"] = clocks
+        res["gpu_launches"] = delta_stack.launches_per_step() * K
+        res["cpu_baseline"] = (cpu_baseline_leg(cfg, case, args.cpu_seconds)
+                               if rank == 0 and world == 1 and not args.no_cpu_baseline else None)
     del g_delta, g_full
     delta_stack.graph = None
     full_stack.graph = None
+    del dc
+    torch.cuda.empty_cache()
+    return res
+
+
+def check_points(cfg, m: int) -> list:
+    """Trajectory steps the oracle checks: the first step, both sides of every drift boundary, the last."""
+    T = cfg.steps
+    pts = {0, T - 1}
+    if cfg.drift_every:
+        for s in range(cfg.drift_every, T, cfg.drift_every):
+            pts.update((s - 1, s))
+    pts = sorted(pts)
+    return pts if m < 0 else pts[:m]
+
+
+def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
+    """The drifting trajectory: every decode step replays one CUDA graph; between steps (untimed)
+    the cache grows by one token per sequence and, every drift_every steps, the planted keys move."""
+    import numpy as np
+    import torch
+    from synth.trajectory import Trajectory
+
+    T = cfg.steps
+    K = min(args.steps, T) if args.steps else T
+    timed_steps = sorted({int(round(i * (T - 1) / max(K - 1, 1))) for i in range(K)}) if K > 1 else [0]
+    checks = check_points(cfg, args.checks) if rank == 0 else []
+    pool = None
+    if checks:
+        from oracle.parallel import OraclePool
+        pool = OraclePool(args.oracle_procs or None)   # spawn-started: safe after CUDA init
+
+    tr = Trajectory(cfg, device=device)
+    dc = tr.dc
+    case0 = tr.case0
+    mk = make_stacks(cfg, case0, dc, args.reduce)
+    stack = mk(cfg.layer_kinds())
+    full_stack = mk(["full"] * cfg.num_layers)
+    tr.prepare(0)
+    step_args = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    g = stack.capture(*step_args)
+    g_full = full_stack.capture(*step_args)
+    gpu = Gpu(device, dist)
+    k2 = max(min(K, 50), 10)
+
+    # ---- at the first step (appending the same token again changes nothing): DELTA vs all-full
+    #      stack, kernel rooflines, per-call breakdown, end to end through the public API
+    us_delta0 = gpu.mean_us(g.replay, k2)
+    us_full0 = gpu.mean_us(g_full.replay, k2)
+    km = kernel_measurements(gpu, cfg, case0, dc, stack, us_full0, k2)
+    e2e = e2e_measure(gpu, cfg, dc, mk, k2)
+    del g_full
+    full_stack.graph = None
+
+    # ---- the trajectory (the headline)
+    sampler = ClockSampler(gpu_index(device))
+    sampler.start()
+    time.sleep(0.3)
+    for _ in range(args.warmup):
+        gpu.flush_l2()
+        g.replay()
+    barrier(dist, device)
+    timed = set(timed_steps)
+    events, pending, gpu_sel, gpu_out = [], [], {}, {}
+    ld = stack.delta_layers
+    for step in range(T):
+        tr.prepare(step)
+        if step in timed:
+            gpu.flush_l2()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(gpu.stream)
+            g.replay()
+            s1.record(gpu.stream)
+            events.append((s0, s1))
+        else:
+            g.replay()
+        if step in checks:
+            cnt = stack.sel_cnt.cpu().numpy()
+            pages = stack.sel_pages.cpu().numpy()
+            outs = dc.out[ld].float().cpu().numpy()
+            for i, l in enumerate(ld):
+                for b in range(cfg.batch):
+                    gpu_sel[(step, l, b)] = pages[i, b, :cnt[i, b]].tolist()
+                    gpu_out[(step, l, b)] = outs[i, b]
+            pending.append(pool.submit([(cfg, step, "delta", l, b) for l in ld for b in range(cfg.batch)]))
+    barrier(dist, device)
+    clocks = sampler.stop()
+    lat = np.array([s.elapsed_time(e) * 1000.0 for s, e in events])
+    us = max_over_ranks(dist, float(lat.mean()), device)
+
+    # ---- the oracle's verdict on the sampled steps
+    check = None
+    if pending:
+        from oracle.checks import selection_ok
+        ok = exact = total = 0
+        worst_abs = worst_rel = 0.0
+        for res in pending:
+            for job, (o_ref, S) in res.get():
+                _, step, _, l, b = job
+                n = int(cfg.contexts(step)[b])
+                good, ex, _ = selection_ok(gpu_sel[(step, l, b)], S, n, cfg.budget_pages, cfg.sink_tokens,
+                                           cfg.recency_tokens, cfg.page_size)
+                ok += int(good)
+                exact += int(ex)
+                total += 1
+                o = gpu_out[(step, l, b)].astype(np.float64)
+                worst_abs = max(worst_abs, float(np.abs(o - o_ref).max()))
+                worst_rel = max(worst_rel, float(np.linalg.norm(o - o_ref) / max(np.linalg.norm(o_ref), 1e-30)))
+        pool.close()
+        check = {"selection_match_rate": round(ok / total, 4), "selections_checked": total,
+                 "selections_exact": exact, "steps_checked": checks,
+                 "rule": "every delta-layer x every sequence at each checked step; a match is the oracle's set, "
+                         "pages swapped only inside a band of scores within 1e-4 relative of the k-th",
+                 "delta_output_max_abs_err": round(worst_abs, 6), "delta_output_max_rel_l2": round(worst_rel, 6)}
+    elif pool is not None:
+        pool.close()
+
+    tok = [attended_tokens(cfg, tr.case_at(s)) for s in (0, T - 1)]
+    n_sparse = cfg.layer_kinds().count("sparse")
+    km["roofline"]["share_of_step"] = round(n_sparse * km["roofline"]["us_per_launch"] / us_delta0, 3)
+    res = {
+        "us_per_step": round(us, 3),
+        "trajectory": {"per_step_us": {"mean": round(float(lat.mean()), 3), "median": round(float(np.median(lat)), 3),
+                                       "p99": round(float(np.percentile(lat, 99)), 3),
+                                       "first": round(float(lat[0]), 3), "last": round(float(lat[-1]), 3)},
+                       "timed_steps": len(timed_steps), "steps_run": T, "oracle_check": check},
+        "step0_us": round(us_delta0, 3), "full_stack_us": round(us_full0, 3),
+        "speedup_vs_full_stack": round(us_full0 / us_delta0, 3),
+        "attended_token_reduction": round(statistics.mean(t[1] / t[0] for t in tok), 3),
+        "speedup_note": "DELTA and all-full stacks both timed at the trajectory's first step",
+    }
+    res.update(km)
+    res["e2e"] = e2e
+    res["clocks"] = clocks
+    res["gpu_launches"] = stack.launches_per_step() * len(timed_steps)
+    res["cpu_baseline"] = (cpu_baseline_leg(cfg, case0, args.cpu_seconds)
+                           if rank == 0 and world == 1 and not args.no_cpu_baseline else None)
+    del g
+    stack.graph = None
+    del tr, dc
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    import torch
+    from synth import configs as C
+    dist, rank, world, local = dist_init()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = C.CONFIGS[args.config]
+    if cfg.steps > 1:
+        r = run_trajectory(args, cfg, dist, rank, world, device)
+        K = r["trajectory"]["timed_steps"]
+    else:
+        r = run_static(args, cfg, dist, rank, world, device)
+        K = args.steps if args.steps else 200
+    also = {}
+    if not args.no_extra and world == 1 and args.config == 5:
+        ea = parse(["--steps", "20", "--warmup", "3", "--reduce", args.reduce])
+        for c in (C.LLAMA8B_64K, C.QWEN7B_8K):
+            x = run_static(ea, c, dist, rank, world, device, headline=False)
+            also[c.name] = {key: x[key] for key in ("us_per_step", "full_stack_us", "speedup_vs_full_stack",
+                                                    "attended_token_reduction")}
+            for key in ("roofline", "roofline_full_layer", "roofline_delta_layer"):
+                also[c.name][key] = {f: x[key][f] for f in ("frac", "achieved", "us_per_launch", "alg_bytes_per_launch")}
+    us = r.pop("us_per_step")
+    if rank == 0:
+        line = {"metric": METRIC, "value": us, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+                "ms_per_step": round(us / 1000, 6), "higher_is_better": False, "scaling": "weak",
+                "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+                "config": config_dict(cfg, args.reduce, world)}
+        line.update(r)
+        if also:
+            line["also"] = also
+        print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
 
@@ -623,7 +794,6 @@ def delta_placement(num_layers: int, m: int) -> list:
 def run_delta_sweep(args, cfg, counts):
     """Decode-step time against the number of delta-layers on one workload (one JSON line)."""
     import torch
-    from long_context_layer_b200.stack import DeltaStack
     from synth.case import Case
     from synth.gpu import DeviceCase
 
@@ -631,28 +801,15 @@ def run_delta_sweep(args, cfg, counts):
     torch.cuda.set_device(device)
     case = Case(cfg)
     dc = DeviceCase(case, device=device, prefill="append")
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
-    flush_rd = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
-    args_step = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    gpu = Gpu(device)
+    step_args = (dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    mk = make_stacks(cfg, case, dc, args.reduce)
+    K = args.steps if args.steps else 50
 
     def time_kinds(kinds):
-        st = DeltaStack(kinds, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, dc.dtype, dc.indptr, dc.indices,
-                        dc.kv_len, case.max_pages_per_seq, dc.num_phys_pages, cfg.budget_pages, cfg.sink_tokens,
-                        cfg.recency_tokens)
-        g = st.capture(*args_step)
-        ts = []
-        for i in range(args.warmup + args.steps):
-            flush.fill_(1)
-            flush_rd.sum()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-            e1.synchronize()
-            if i >= args.warmup:
-                ts.append(e0.elapsed_time(e1) * 1000.0)
+        st = mk(kinds)
+        g = st.capture(*step_args)
+        ts = gpu.timed(g.replay, K, args.warmup)
         del g
         st.graph = None
         return statistics.median(ts)
@@ -672,7 +829,8 @@ def run_delta_sweep(args, cfg, counts):
     print(json.dumps({"metric": "us_per_decode_step_vs_delta_layer_count", "unit": "us/step",
                       "config": {"workload": cfg.name, "layers": L, "batch": cfg.batch,
                                  "context": int(case.n.max())},
-                      "full_stack_us": round(full_us, 3), "steps": args.steps, "warmup": args.warmup,
+                      "kernel_sources_sha256": kernel_source_hash(),
+                      "full_stack_us": round(full_us, 3), "steps": K, "warmup": args.warmup,
                       "points": points}), flush=True)
 
 
@@ -685,11 +843,8 @@ def main():
         run_reference(args)
         return
     from synth import configs as C
-    cfg = C.CONFIGS[args.config]
     if args.delta_sweep:
-        run_delta_sweep(args, cfg, [int(x) for x in args.delta_sweep.split(",")])
-    elif cfg.steps > 1:
-        run_trajectory(args, cfg)
+        run_delta_sweep(args, C.CONFIGS[args.config], [int(x) for x in args.delta_sweep.split(",")])
     else:
         run_ours(args)
 

@@ -189,7 +189,12 @@ delta_status delta_full_attn_noalloc(const delta_desc* desc, const delta_page_ta
  * pages and the budget_pages best remaining pages, written ascending to
  * sel_pages[b][0..sel_cnt[b]).  page_scores may be NULL; when given, S is written
  * for j < ceil(kv_len[b]/page_size).  sel_stride must be >= delta_sel_capacity().
- * max_pages_per_seq must be <= 32768 here. */
+ * max_pages_per_seq must be <= 32768 here.
+ * HEAD_SUM runs as one kernel: the last CTA to finish among a sequence's CTAs scores
+ * its pages and selects them (arrival counters in the workspace; no CTA waits).
+ * HEAD_MAX adds a second kernel that scores every token.  The workspace's counters
+ * return to zero at the end of every call; after a call that failed to launch or
+ * was cut short, re-initialise the workspace (delta_workspace_init). */
 delta_status delta_select_attn(const delta_desc* desc, const delta_page_table* pt,
                                const delta_select_params* sp,
                                const void* q, const void* k_pool, const void* v_pool, void* o,

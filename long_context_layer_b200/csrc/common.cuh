@@ -331,7 +331,14 @@ __device__ __forceinline__ void seq_count(const P& p, int b, SeqExtent& ex) {
 // so other CTAs of the cluster may push into it while this CTA is still streaming pages).  Its
 // first 16 bytes hold the mbarrier that counts the bytes pushed into it.
 template <int D>
-constexpr int recv_floats() { return 4 + kMaxGroup * D + 16 * 4 + 16 * kMaxGroup * 2 + kMaxGroup * 2; }
+constexpr int recv_floats() { return 4 + kMaxGroup * D + 16 * 4 + 16 * kMaxGroup * 4 + kMaxGroup * 2; }
+
+// Per-CTA states [C][G][4] inside a cluster's merge receive area (after its barrier and the C slices).
+template <int D, int G>
+__device__ __forceinline__ const float* merge_recv_states(const float* recv, int C) {
+    const int chunk = (((G * D + C - 1) / C) + 3) & ~3;
+    return recv + 4 + C * chunk;
+}
 
 // Kernel prologue of the cluster merge, all threads, before the wait for the previous kernel:
 // thread 0 initialises this CTA's receive barrier, then one cluster barrier makes every CTA's
@@ -375,9 +382,13 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
     const int chunk = (((total + C - 1) / C) + 3) & ~3;
     uint64_t* rbar = reinterpret_cast<uint64_t*>(recv);
     recv += 4;
-    float* recv_ml = recv + C * chunk;                                             // [C][G][2]
+    // [C][G][4]: each CTA's (max, sum) per head, and on delta-layers also the state over the exact
+    // fp32 page terms, from which every CTA forms the page scores' per-head normalisers itself
+    float* recv_ml = recv + C * chunk;
+    const bool delta = p.mode == kModeDelta;
     const int e0 = rank * chunk, e1 = min(e0 + chunk, total);                      // this CTA's slice
-    if (tid == 0) mbar_expect_tx(rbar, uint32_t(C) * (uint32_t(max(e1 - e0, 0)) * 4u + uint32_t(G) * 8u));
+    if (tid == 0)
+        mbar_expect_tx(rbar, uint32_t(C) * (uint32_t(max(e1 - e0, 0)) * 4u + uint32_t(G) * (delta ? 16u : 8u)));
     auto part_max = [&](const float* ml, int h) {
         float M = -INFINITY;
 #pragma unroll
@@ -395,15 +406,17 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
         const int j = tid / G, h = tid % G;
         const float M = part_max(mml, h);
         const float L = part_sum(mml, h, M);
-        st_async(cluster_addr(recv_ml + (rank * G + h) * 2, j), make_float2(M, L), cluster_addr(rbar, j));
-        if (j == 0 && p.split_ml != nullptr) {   // the selection combines its per-head totals from these
-            float Md = M, Ld = L;
-            if (dml != nullptr) {
-                Md = part_max(dml, h);
-                Ld = part_sum(dml, h, Md);
-            }
-            p.split_ml[(size_t(b) * Hq + h0 + h) * p.num_splits + blockIdx.x] = make_float2(Md, Ld);
+        float Md = M, Ld = L;
+        if (dml != nullptr) {
+            Md = part_max(dml, h);
+            Ld = part_sum(dml, h, Md);
         }
+        if (delta)
+            st_async(cluster_addr(recv_ml + (rank * G + h) * 4, j), make_float4(M, L, Md, Ld), cluster_addr(rbar, j));
+        else
+            st_async(cluster_addr(recv_ml + (rank * G + h) * 4, j), make_float2(M, L), cluster_addr(rbar, j));
+        if (j == 0 && p.split_ml != nullptr)   // the selection combines its per-head totals from these
+            p.split_ml[(size_t(b) * Hq + h0 + h) * p.num_splits + blockIdx.x] = make_float2(Md, Ld);
     }
     for (int q4 = tid; q4 * 4 < total; q4 += nthr) {
         const int idx = q4 * 4, h = idx / D, d = idx % D;    // D is a multiple of 4: one head per group
@@ -429,12 +442,12 @@ __device__ __forceinline__ void merge_epilogue(const DecodeParams& p, unsigned c
     for (int e = e0 + tid; e < e1; e += nthr) {
         const int h = e / D, d = e % D;
         float M = -INFINITY;
-        for (int j = 0; j < C; ++j) M = fmaxf(M, recv_ml[(j * G + h) * 2]);
+        for (int j = 0; j < C; ++j) M = fmaxf(M, recv_ml[(j * G + h) * 4]);
         const float mu = (M == -INFINITY) ? 0.f : M;
         float L = 0.f, acc = 0.f;
         for (int j = 0; j < C; ++j) {
-            const float w = exp2_approx(recv_ml[(j * G + h) * 2] - mu);
-            L = fmaf(w, recv_ml[(j * G + h) * 2 + 1], L);
+            const float w = exp2_approx(recv_ml[(j * G + h) * 4] - mu);
+            L = fmaf(w, recv_ml[(j * G + h) * 4 + 1], L);
             acc = fmaf(w, recv[j * chunk + (e - e0)], acc);
         }
         if (nC == 1) {

@@ -74,7 +74,7 @@ struct MmaSmem {
 };
 
 template <int D, int G, int STAGES, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodeParams p,
+__global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeParams p,
                                                               const __grid_constant__ CUtensorMap tmap_k,
                                                               const __grid_constant__ CUtensorMap tmap_v) {
     using S = MmaSmem<D, STAGES, WARPS>;
@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_mma_kernel(const DecodePara
         p, smem, mo0, mo0 + kMaxGroup * kRow, recv, b, g, kPart, kPart,
         (p.mode == kModeDelta) ? mo0 + kMaxGroup * kRow + kMaxGroup * 2 : nullptr);
     // delta-layers scoring with HEAD_SUM: page scores and the selection, in the stage area
-    if (p.fuse_select) select_tail<WARPS * 32, G>(p, smem, S::kStages, b, g, ex.n, ex.N);
+    if (p.fuse_select) select_tail<WARPS * 32, G, D>(p, smem, S::kStages, recv, b, g, ex.n, ex.N);
 }
 
 }  // namespace delta

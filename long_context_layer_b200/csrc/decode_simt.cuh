@@ -20,7 +20,7 @@ struct DecodeSmem {
 };
 
 template <typename T, int D, int G, int STAGES>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
     using S = DecodeSmem<T, D, STAGES>;
     constexpr int DS = D / 16;          // dimensions per lane
     constexpr int GP = pad_group(G);    // group padded to a power of two
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     __syncthreads();
     merge_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, recv, b, g, kMaxGroup * D, kMaxGroup * 2);
     // delta-layers scoring with HEAD_SUM: page scores and the selection, in the stage area
-    if (p.fuse_select) select_tail<kThreads, G>(p, smem, S::kMain, b, g, ex.n, ex.N);
+    if (p.fuse_select) select_tail<kThreads, G, D>(p, smem, S::kMain, recv, b, g, ex.n, ex.N);
 }
 
 }  // namespace delta

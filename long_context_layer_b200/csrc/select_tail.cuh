@@ -8,12 +8,14 @@
 // = sum_h 2^(lse_hj - c_h), with lse_hj the log2-sum-exp of head h's base-2 logits on page j
 // (written by the decode loop) and c_h that head's log2-sum-exp over the whole context.
 //
-// No CTA waits for another.  Every CTA of the grid takes a ticket on its (sequence, KV head)
-// unit once its page terms and split state are visible; the unit's last CTA forms c_h of the
-// unit's G heads from the splits' states and writes the unit's share of every page score; it
-// then takes a ticket on its sequence, and the sequence's last unit sums the KV heads' shares
-// (fixed order: deterministic), finds the k-th largest candidate score by an adaptive-range
-// radix select and writes the ascending selection.
+// No CTA waits for another.  When a (sequence, KV head) unit is one cluster, the output merge has
+// already given every CTA every split's state of the unit's heads, so each CTA forms c_h itself,
+// writes its own pages' share of the scores (the sum over the unit's G heads) and takes one
+// ticket on its sequence.  When a unit spans several clusters, each CTA takes a ticket on its
+// unit first, and the unit's last CTA forms c_h from the splits' states in the workspace and
+// writes the unit's shares.  The last CTA of the sequence sums the KV heads' shares (fixed order:
+// deterministic), finds the k-th largest candidate score by an adaptive-range radix select and
+// writes the ascending selection.
 #pragma once
 
 #include "common.cuh"
@@ -52,103 +54,66 @@ __device__ __forceinline__ uint64_t block_scan_u64(uint64_t x, uint64_t* sums, u
     return sums[warp] + incl - x;
 }
 
-// Every thread of the CTA calls this after the output merge.  smem: the kernel's page-stage area,
-// idle by now (free_bytes long, 16-byte aligned).  n, N: the sequence's tokens and pages.
-template <int NTHR, int G>
-__device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char* smem, size_t free_bytes, int b, int g,
-                                         int n, int N) {
+// What the sequence's last CTA needs (passed by value to the non-inlined final stage).
+struct SelectFinal {
+    const float* unit_scores;   // [B][Hkv][max_pages]
+    uint32_t* keys;             // [B][max_pages]
+    float* page_scores;         // [B][max_pages] or null
+    int32_t* sel_cnt;
+    int32_t* sel_pages;
+    int32_t sel_stride, max_pages, num_kv_heads, budget_pages, sink_tokens, recency_tokens;
+};
+
+// Takes a ticket on `counter`; true in every thread of the CTA that arrives `expected`-th (which
+// also resets the counter for the next launch).  The CTA's earlier global writes are visible to
+// that CTA first.
+__device__ __forceinline__ bool arrive_last(int* counter, int expected, uint32_t* s_flag) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int t = atomicAdd(counter, 1);
+        const uint32_t last = (t == expected - 1) ? 1u : 0u;
+        if (last) *counter = 0;
+        *s_flag = last;
+    }
+    __syncthreads();
+    const bool last = *s_flag != 0u;
+    if (last) __threadfence();
+    return last;
+}
+
+// Steps of the sequence's last CTA: page scores and their order keys, the threshold key T and the
+// number of keys equal to T to take, then the ascending compaction.  smem: free_bytes of idle
+// shared memory (16-byte aligned).
+template <int NTHR>
+__device__ __noinline__ void select_final(const SelectFinal a, unsigned char* smem, size_t free_bytes, int b, int n,
+                                          int N) {
     constexpr int W = NTHR / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, S = p.num_splits, h0 = g * G;
-    const size_t maxp = size_t(p.max_pages);
-
+    const size_t maxp = size_t(a.max_pages);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem);      // [256]
     uint32_t* list = hist + 256;                              // [kTailList]
     uint64_t* sums = reinterpret_cast<uint64_t*>(list + kTailList);   // [W + 1]
-    float* s_c = reinterpret_cast<float*>(sums + W + 1);      // [kMaxGroup] per-head normalisers
-    uint32_t* s_u = reinterpret_cast<uint32_t*>(s_c + kMaxGroup);     // [8] flags and broadcasts
+    uint32_t* s_u = reinterpret_cast<uint32_t*>(sums + W + 1);        // [8] broadcasts
     uint32_t* s_wmin = s_u + 8;                               // [W]
     uint32_t* s_wmax = s_wmin + W;                            // [W]
-    constexpr size_t kScratch = ((256 + kTailList) * 4 + (W + 1) * 8 + kMaxGroup * 4 + 8 * 4 + 2 * W * 4 + 15) & ~size_t(15);
-    uint32_t* skeys = reinterpret_cast<uint32_t*>(smem + kScratch);
+    constexpr size_t kScratch = ((256 + kTailList) * 4 + (W + 1) * 8 + 8 * 4 + 2 * W * 4 + 15) & ~size_t(15);
     const int key_cap = int((free_bytes - kScratch) / 4);
+    uint32_t* keys = (N <= key_cap) ? reinterpret_cast<uint32_t*>(smem + kScratch) : a.keys + size_t(b) * maxp;
 
-    // 1. this CTA's page terms (page_lse) and split state (split_ml) are visible: arrive at the unit
-    __threadfence();
-    __syncthreads();   // also: no thread still reads the merge records in the stage area
-    if (tid == 0) {
-        const int t = atomicAdd(&p.unit_tickets[b * Hkv + g], 1);
-        const uint32_t last = (t == S - 1) ? 1u : 0u;
-        if (last) p.unit_tickets[b * Hkv + g] = 0;   // ready for the next launch
-        s_u[0] = last;
-    }
-    __syncthreads();
-    if (!s_u[0]) return;
-    __threadfence();
-
-    // 2. c_h of the unit's heads: log2 of the sum of 2^(m) l over the splits' (max, sum) states
-    for (int h = warp; h < G; h += W) {
-        const float2* ps = p.split_ml + (size_t(b) * Hq + h0 + h) * S;
-        float M = -INFINITY, Z = 0.f;
-        for (int base = 0; base < S; base += 32) {
-            const float2 v = (base + lane < S) ? __ldcg(ps + base + lane) : make_float2(-INFINITY, 0.f);
-            float Mr = v.x;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
-            const float Mn = fmaxf(M, Mr);
-            const float mu = (Mn == -INFINITY) ? 0.f : Mn;
-            float z = (v.y > 0.f) ? v.y * exp2_approx(v.x - mu) : 0.f;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            Z = Z * exp2_approx(M - mu) + z;
-            M = Mn;
-        }
-        // no token of the head: every page term is 2^(-inf) = 0
-        if (lane == 0) s_c[h] = (Z > 0.f) ? M + log2_approx(Z) : INFINITY;
-    }
-    __syncthreads();
-
-    // 3. the unit's share of every page score: sum over its G heads of 2^(lse_hj - c_h)
-    {
-        float* us = p.unit_scores + (size_t(b) * Hkv + g) * maxp;
-        const float* pl = p.page_lse + (size_t(b) * Hq + h0) * maxp;
-        for (int j = tid; j < N; j += NTHR) {
-            float v[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) v[h] = __ldcg(pl + size_t(h) * maxp + j);
-            float sc = 0.f;
-#pragma unroll
-            for (int h = 0; h < G; ++h) sc += exp2_approx(v[h] - s_c[h]);
-            us[j] = sc;
-        }
-    }
-
-    // 4. the unit's shares are visible: arrive at the sequence
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const int t = atomicAdd(&p.seq_tickets[b], 1);
-        const uint32_t last = (t == Hkv - 1) ? 1u : 0u;
-        if (last) p.seq_tickets[b] = 0;
-        s_u[0] = last;
-    }
-    __syncthreads();
-    if (!s_u[0]) return;
-    __threadfence();
-
-    // 5. page scores (the KV heads' shares summed in head order) and their order keys; the range of
-    //    the candidate keys (pages neither sink nor recency)
-    const int sinkP = min((min(p.sink_tokens, n) + kPage - 1) / kPage, N);
-    const int recStart = (p.recency_tokens > 0) ? min(max(n - p.recency_tokens, 0) / kPage, N) : N;
-    const int k = p.budget_pages;
+    // 1. page scores (the KV heads' shares summed in head order), order keys, candidate key range
+    //    (candidates: pages neither sink nor recency)
+    const int sinkP = min((min(a.sink_tokens, n) + kPage - 1) / kPage, N);
+    const int recStart = (a.recency_tokens > 0) ? min(max(n - a.recency_tokens, 0) / kPage, N) : N;
+    const int k = a.budget_pages;
     const bool take_all = max(recStart - sinkP, 0) <= k;
     const bool radix = !take_all && k > 0;
-    uint32_t* keys = (N <= key_cap) ? skeys : p.keys + size_t(b) * maxp;
+    const float* us = a.unit_scores + size_t(b) * a.num_kv_heads * maxp;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     for (int j = tid; j < N; j += NTHR) {
         float sc = 0.f;
-        for (int u = 0; u < Hkv; ++u) sc += __ldcg(p.unit_scores + (size_t(b) * Hkv + u) * maxp + j);
-        if (p.page_scores != nullptr) p.page_scores[size_t(b) * maxp + j] = sc;
+        for (int u = 0; u < a.num_kv_heads; ++u) sc += __ldcg(us + size_t(u) * maxp + j);
+        if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
         const uint32_t key = order_key(sc);
         keys[j] = key;
         if (j >= sinkP && j < recStart) {
@@ -164,7 +129,7 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
     }
     __syncthreads();
 
-    // 6. threshold T and the number of keys equal to T to take (lowest page index first).  Each
+    // 2. threshold T and the number of keys equal to T to take (lowest page index first).  Each
     //    pass buckets the keys of [lo, lo + span] into 256 buckets of width 2^sh, finds the bucket
     //    holding the kk-th largest and narrows the range to it (span shrinks by 2^8 a pass, so at
     //    most four passes); once the bucket holds at most kTailList keys they are ranked exactly.
@@ -269,7 +234,7 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
         }
     }
 
-    // 7. ascending compaction of sink U recency U {key > T} U {the first `need` keys == T}: each
+    // 3. ascending compaction of sink U recency U {key > T} U {the first `need` keys == T}: each
     //    thread owns a contiguous run of pages; one scan of the packed (equal, taken) counts gives
     //    every thread its output position
     const int per = (N + NTHR - 1) / NTHR;
@@ -290,7 +255,7 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
     const uint32_t eq_tot = uint32_t(tot), take_tot = uint32_t(tot >> 32);
     uint32_t pos = take_rank + min(need, eq_rank);
     uint32_t eq_seen = eq_rank;
-    int32_t* out = p.sel_pages_out + size_t(b) * p.sel_stride_out;
+    int32_t* out = a.sel_pages + size_t(b) * a.sel_stride;
     for (int j = jb; j < je; ++j) {
         bool take;
         if (take_all || j < sinkP || j >= recStart) {
@@ -302,11 +267,99 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
             take = key > T || (key == T && eq_seen++ < need);
         }
         if (take) {
-            if (pos < uint32_t(p.sel_stride_out)) out[pos] = j;
+            if (pos < uint32_t(a.sel_stride)) out[pos] = j;
             ++pos;
         }
     }
-    if (tid == 0) p.sel_cnt_out[b] = int(min(take_tot + min(need, eq_tot), uint32_t(p.sel_stride_out)));
+    if (tid == 0) a.sel_cnt[b] = int(min(take_tot + min(need, eq_tot), uint32_t(a.sel_stride)));
+}
+
+// Every thread of the CTA calls this after the output merge.  smem: the kernel's page-stage area,
+// idle by now (free_bytes long, 16-byte aligned); recv: the merge's receive area; n, N: the
+// sequence's tokens and pages.
+template <int NTHR, int G, int D>
+__device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char* smem, size_t free_bytes,
+                                            const float* recv, int b, int g, int n, int N) {
+    constexpr int W = NTHR / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, S = p.num_splits, h0 = g * G;
+    const size_t maxp = size_t(p.max_pages);
+    float* s_c = reinterpret_cast<float*>(smem);               // [kMaxGroup] per-head normalisers
+    uint32_t* s_flag = reinterpret_cast<uint32_t*>(s_c + kMaxGroup);
+    const float* pl = p.page_lse + (size_t(b) * Hq + h0) * maxp;
+    float* us = p.unit_scores + (size_t(b) * Hkv + g) * maxp;
+    // the unit's share of page j's score: the sum over its G heads of 2^(lse_hj - c_h)
+    auto share = [&](int j) {
+        float v[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) v[h] = __ldcg(pl + size_t(h) * maxp + j);
+        float sc = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) sc += exp2_approx(v[h] - s_c[h]);
+        return sc;
+    };
+    // c_h = log2 of the sum over states of l * 2^m (no token of the head: +inf, every term 0)
+    auto norm = [](float M, float Z) { return (Z > 0.f) ? M + log2_approx(Z) : INFINITY; };
+
+    if (p.num_clusters == 1) {
+        // every state of the unit is in this CTA's receive area: c_h here, then this CTA's pages
+        const int C = S;
+        const float* st = merge_recv_states<D, G>(recv, C);   // [C][G][4]: (m, l) then the fp32-term (m, l)
+        __syncthreads();   // no thread still reads the merge records in the stage area
+        if (tid < G) {
+            float M = -INFINITY;
+            for (int j = 0; j < C; ++j) M = fmaxf(M, st[(j * G + tid) * 4 + 2]);
+            const float mu = (M == -INFINITY) ? 0.f : M;
+            float Z = 0.f;
+            for (int j = 0; j < C; ++j) {
+                const float l = st[(j * G + tid) * 4 + 3];
+                if (l > 0.f) Z = fmaf(l, exp2_approx(st[(j * G + tid) * 4 + 2] - mu), Z);
+            }
+            s_c[tid] = norm(M, Z);
+        }
+        __syncthreads();
+        const int i0 = blockIdx.x * p.items_per_split, i1 = min(i0 + p.items_per_split, N);
+        for (int j = i0 + tid; j < i1; j += NTHR) us[j] = share(j);
+        if (!arrive_last(p.seq_tickets + b, Hkv * S, s_flag)) return;
+    } else {
+        // the unit's last CTA forms c_h from the splits' states and writes the unit's shares
+        if (!arrive_last(p.unit_tickets + b * Hkv + g, S, s_flag)) return;
+        for (int h = warp; h < G; h += W) {
+            const float2* ps = p.split_ml + (size_t(b) * Hq + h0 + h) * S;
+            float M = -INFINITY, Z = 0.f;
+            for (int base = 0; base < S; base += 32) {
+                const float2 v = (base + lane < S) ? __ldcg(ps + base + lane) : make_float2(-INFINITY, 0.f);
+                float Mr = v.x;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
+                const float Mn = fmaxf(M, Mr);
+                const float mu = (Mn == -INFINITY) ? 0.f : Mn;
+                float z = (v.y > 0.f) ? v.y * exp2_approx(v.x - mu) : 0.f;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                Z = Z * exp2_approx(M - mu) + z;
+                M = Mn;
+            }
+            if (lane == 0) s_c[h] = norm(M, Z);
+        }
+        __syncthreads();
+        for (int j = tid; j < N; j += NTHR) us[j] = share(j);
+        if (!arrive_last(p.seq_tickets + b, Hkv, s_flag)) return;
+    }
+    SelectFinal a;
+    a.unit_scores = p.unit_scores;
+    a.keys = p.keys;
+    a.page_scores = p.page_scores;
+    a.sel_cnt = p.sel_cnt_out;
+    a.sel_pages = p.sel_pages_out;
+    a.sel_stride = p.sel_stride_out;
+    a.max_pages = p.max_pages;
+    a.num_kv_heads = Hkv;
+    a.budget_pages = p.budget_pages;
+    a.sink_tokens = p.sink_tokens;
+    a.recency_tokens = p.recency_tokens;
+    __syncthreads();   // s_c and s_flag are about to be overwritten by the final stage's scratch
+    select_final<NTHR>(a, smem, free_bytes, b, n, N);
 }
 
 }  // namespace delta

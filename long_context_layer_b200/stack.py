@@ -68,7 +68,9 @@ class DeltaStack:
 
     # ------------------------------------------------------------------ one step
     def launches_per_step(self, append: bool = True) -> int:
-        per = {FULL: 1, DELTA: 2, SPARSE: 1}
+        # a delta-layer scoring with HEAD_SUM selects its pages inside its decode kernel; HEAD_MAX
+        # adds a selection kernel
+        per = {FULL: 1, DELTA: 1 if self.sp.reduce == N.DELTA_HEAD_SUM else 2, SPARSE: 1}
         return sum(per[k] for k in self.kinds) + (1 if append else 0)
 
     def step(self, q, k_new, v_new, k_pools, v_pools, out, append: bool = True, stream: int | None = None):

@@ -54,3 +54,25 @@ def test_sweep_placement_spreads_delta_layers_from_layer_2():
             pl = bench.delta_placement(L, m)
             assert pl[0] == 2 and len(pl) == m and pl == sorted(set(pl)) and pl[-1] < L
         assert bench.delta_placement(L, L - 2) == list(range(2, L))   # every layer from 2: the full stack
+
+
+def test_both_arms_report_the_same_config_dict():
+    import bench
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "1",
+                        "--steps", "2", "--warmup", "1", "--cpu-seconds", "1"], capture_output=True, text=True,
+                       timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.strip().startswith("{")][0])
+    # the GPU arm prints bench.config_dict(cfg, reduce, world) for the same workload
+    assert d["config"] == json.loads(json.dumps(bench.config_dict(C.TINY, "sum", 1)))
+    assert d["steps"] == 2 and d["warmup"] == 1
+
+
+def test_trajectory_check_points_straddle_every_drift_boundary():
+    import bench
+    pts = bench.check_points(C.DRIFT_48L, -1)
+    assert pts[0] == 0 and pts[-1] == 999 and len(pts) == 20   # 0, 99, 100, ..., 899, 900, 999
+    for s in range(100, 1000, 100):
+        assert s - 1 in pts and s in pts
+    assert bench.check_points(C.DRIFT_48L, 3) == [0, 99, 100]
+    assert bench.check_points(C.DRIFT_48L, 0) == []
