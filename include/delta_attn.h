@@ -235,6 +235,19 @@ delta_status delta_sparse_attn_settled(const delta_desc* desc, const delta_page_
 delta_status delta_layer_shift(const delta_page_table* pt, const float* scores_a, const float* scores_b,
                                float* shift_out, void* stream);
 
+/* Delta-layer placement from calibration shifts (a HOST function: plain host arrays, no GPU
+ * work).  shift[l] is the averaged shift between layers l-1 and l (delta_layer_shift, averaged by
+ * the caller over steps and inputs).  The page fixes the first delta-layer (layer 2) and asks
+ * for the rest at layers of large shift spread over the depth (ai.info summary, "Methodology in
+ * Plain English" and "Main Findings", last bullet).  Rule: `first` opens the list; the layers
+ * after it are taken by decreasing shift (equal shifts: lower layer first), each kept only when
+ * at least min_gap layers from every layer already kept, until `count` are kept or none is left.
+ * out_layers (host, room for max(count, 1) entries) receives them ascending, *out_count their
+ * number.  DELTA_ERR_INVALID_ARG for null pointers, num_layers outside 1..4096, first outside
+ * the layers, min_gap < 0 or a NaN shift. */
+delta_status delta_choose_layers(const float* shift, int32_t num_layers, int32_t count, int32_t first,
+                                 int32_t min_gap, int32_t* out_layers, int32_t* out_count);
+
 /* Synchronise `stream`, read and clear the workspace's device error flags.
  * Returns DELTA_OK, DELTA_ERR_BOUNDS (a device-side check failed since the last
  * read) or DELTA_ERR_CUDA.  *flags_out (nullable) receives the raw flag bits:

@@ -7,6 +7,6 @@ the binding fails when the library is missing.
 from . import _native  # noqa: F401  (fails loudly if the library is not built)
 from ._native import (  # noqa: F401
     DELTA_BF16, DELTA_F32, DELTA_HEAD_MAX, DELTA_HEAD_SUM, DeltaDesc, DeltaError, DeltaPageTable,
-    DeltaSelectParams, full_attn, full_attn_noalloc, kv_append, kv_append_layers, layer_shift, read_device_error, sel_capacity, select_attn, sparse_attn, sparse_attn_settled,
+    DeltaSelectParams, choose_layers, full_attn, full_attn_noalloc, kv_append, kv_append_layers, layer_shift, read_device_error, sel_capacity, select_attn, sparse_attn, sparse_attn_settled,
     status_string, workspace_init, workspace_size, workspace_size_reduce,
 )

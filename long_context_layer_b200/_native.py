@@ -28,7 +28,7 @@ EXPORTED = [
     "delta_kv_append_layers",
     "delta_full_attn", "delta_full_attn_noalloc", "delta_select_attn", "delta_sparse_attn",
     "delta_sparse_attn_settled",
-    "delta_layer_shift", "delta_read_device_error",
+    "delta_layer_shift", "delta_choose_layers", "delta_read_device_error",
     "delta_status_string",
 ]
 
@@ -79,6 +79,9 @@ lib.delta_sparse_attn_settled.argtypes = [_D, _PT, _vp, _vp, _i32, _vp, _vp, _vp
 lib.delta_sparse_attn_settled.restype = _i32
 lib.delta_layer_shift.argtypes = [_PT, _vp, _vp, _vp, _vp]
 lib.delta_layer_shift.restype = _i32
+lib.delta_choose_layers.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, _i32, _i32, _i32,
+                                    ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
+lib.delta_choose_layers.restype = _i32
 lib.delta_read_device_error.argtypes = [_vp, ctypes.POINTER(_i32), _vp]
 lib.delta_read_device_error.restype = _i32
 lib.delta_status_string.argtypes = [_i32]
@@ -183,6 +186,17 @@ def sparse_attn_settled(desc, pt, sel_cnt, sel_pages, sel_stride: int, q, k_pool
 def layer_shift(pt, scores_a, scores_b, shift_out, stream: int = 0, check: bool = True) -> int:
     s = lib.delta_layer_shift(ctypes.byref(pt), ptr(scores_a), ptr(scores_b), ptr(shift_out), stream)
     return _check(s, "delta_layer_shift") if check else s
+
+
+def choose_layers(shift, count: int, first: int = 2, min_gap: int = 2) -> list:
+    """delta_choose_layers on a host sequence of per-layer shifts; returns the ascending layer ids."""
+    vals = [float(x) for x in shift]
+    arr = (ctypes.c_float * len(vals))(*vals)
+    out = (_i32 * max(count, 1))()
+    n = _i32(0)
+    _check(lib.delta_choose_layers(arr, len(vals), count, first, min_gap, out, ctypes.byref(n)),
+           "delta_choose_layers")
+    return [int(out[i]) for i in range(n.value)]
 
 
 def read_device_error(workspace, stream: int = 0) -> tuple:

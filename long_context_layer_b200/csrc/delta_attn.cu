@@ -824,6 +824,43 @@ delta_status delta_layer_shift(const delta_page_table* pt, const float* scores_a
                       scores_a, scores_b, pt->page_indptr, pt->kv_len, pt->max_pages_per_seq, shift_out);
 }
 
+delta_status delta_choose_layers(const float* shift, int32_t num_layers, int32_t count, int32_t first,
+                                 int32_t min_gap, int32_t* out_layers, int32_t* out_count) {
+    if (shift == nullptr || out_layers == nullptr || out_count == nullptr) return DELTA_ERR_INVALID_ARG;
+    if (num_layers <= 0 || num_layers > 4096 || first < 0 || first >= num_layers || min_gap < 0)
+        return DELTA_ERR_INVALID_ARG;
+    for (int32_t l = 0; l < num_layers; ++l)
+        if (!(shift[l] == shift[l])) return DELTA_ERR_INVALID_ARG;   // NaN has no order
+    int32_t n = 0;
+    out_layers[n++] = first;
+    // candidates after `first` by decreasing shift, equal shifts lower layer first; a candidate is
+    // kept when at least min_gap layers away from every kept layer
+    bool used[4096] = {false};
+    while (n < count) {
+        int32_t best = -1;
+        for (int32_t l = first + 1; l < num_layers; ++l) {
+            if (used[l]) continue;
+            if (best < 0 || shift[l] > shift[best]) best = l;
+        }
+        if (best < 0) break;
+        used[best] = true;
+        bool far = true;
+        for (int32_t i = 0; i < n; ++i) {
+            const int32_t d = best > out_layers[i] ? best - out_layers[i] : out_layers[i] - best;
+            if (d < min_gap) far = false;
+        }
+        if (far) out_layers[n++] = best;
+    }
+    for (int32_t i = 1; i < n; ++i)   // ascending
+        for (int32_t j = i; j > 0 && out_layers[j - 1] > out_layers[j]; --j) {
+            const int32_t t = out_layers[j];
+            out_layers[j] = out_layers[j - 1];
+            out_layers[j - 1] = t;
+        }
+    *out_count = n;
+    return DELTA_OK;
+}
+
 delta_status delta_read_device_error(void* workspace, int32_t* flags_out, void* stream) {
     if (workspace == nullptr) return DELTA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -140,19 +140,6 @@ class DeltaStack:
 
 
 def choose_delta_layers(shift, count: int, first: int = 2, min_gap: int = 2) -> list:
-    """Delta-layer placement from per-layer shifts (shift[l]: between layers l-1 and l).
-
-    Layer `first` opens the list (DELTA places its first delta-layer at layer 2; ai.info
-    summary, "Methodology in Plain English"); further layers are added by decreasing shift
-    (equal shifts: lower layer first) when at least `min_gap` layers from every layer already
-    in the list, so large shifts are covered without clustering in depth.
-    """
-    shift = [float(x) for x in shift]
-    chosen = [first]
-    order = sorted(range(first + 1, len(shift)), key=lambda l: (-shift[l], l))
-    for l in order:
-        if len(chosen) >= count:
-            break
-        if min(abs(l - c) for c in chosen) >= min_gap:
-            chosen.append(l)
-    return sorted(chosen)
+    """Delta-layer placement from per-layer shifts (shift[l]: between layers l-1 and l), computed by
+    the library's host function delta_choose_layers (the rule is stated in include/delta_attn.h)."""
+    return N.choose_layers(shift, count, first, min_gap)

@@ -129,7 +129,7 @@ def test_empty_batch_is_a_no_op(L):
 
 
 def test_stack_placement_rule_matches_the_oracle():
-    # the product's delta-layer placement (restated in stack.py) equals the oracle's on random shifts,
+    # the library's delta-layer placement (delta_choose_layers, a host function) equals the oracle's on random shifts,
     # ties included
     import numpy as np
     from oracle import delta_oracle as O
@@ -142,3 +142,17 @@ def test_stack_placement_rule_matches_the_oracle():
         count = int(r.integers(1, 6))
         gap = int(r.integers(1, 4))
         assert choose_delta_layers(shift, count, min_gap=gap) == O.choose_delta_layers(shift, count, min_gap=gap)
+
+
+def test_choose_layers_rejects_bad_arguments(L):
+    import ctypes
+    from long_context_layer_b200 import _native as N
+    shift = (ctypes.c_float * 4)(0, 0, 0.5, float("nan"))
+    out = (ctypes.c_int32 * 4)()
+    n = ctypes.c_int32(0)
+    assert N.lib.delta_choose_layers(shift, 4, 2, 2, 1, out, ctypes.byref(n)) == N.DELTA_ERR_INVALID_ARG   # NaN
+    ok = (ctypes.c_float * 4)(0, 0, 0.5, 0.7)
+    assert N.lib.delta_choose_layers(ok, 4, 2, 4, 1, out, ctypes.byref(n)) == N.DELTA_ERR_INVALID_ARG     # first
+    assert N.lib.delta_choose_layers(ok, 4, 2, 2, -1, out, ctypes.byref(n)) == N.DELTA_ERR_INVALID_ARG    # gap
+    assert N.lib.delta_choose_layers(ok, 4, 3, 2, 1, out, ctypes.byref(n)) == N.DELTA_OK
+    assert [out[i] for i in range(n.value)] == [2, 3]        # only two layers after layer 1
