@@ -394,13 +394,17 @@ int max_active_clusters(const void* func, size_t smem, int cluster, int threads)
 // units * clusters all fit in one wave; ties go to the larger cluster (fewer cross-cluster
 // partials).  Long sequences thus keep ~one wave of CTAs even where large clusters do not pack
 // into the GPCs.
-SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items) {
+// one_cluster_per_unit: delta-layers that select their pages at the end of the decode keep every
+// (sequence, KV head) unit in one cluster, so each CTA gets the unit's per-head normalisers from the
+// cluster merge (a unit spread over several clusters needs a second arrival stage).
+SplitPlan fit_plan(SplitPlan pl, int dtype, int D, int G, int units, int items, bool one_cluster_per_unit = false) {
     const int s = pl.splits();
     // Clusters meet through the workspace only when each gets at least 256 pages (and the unit has
     // more than 512): below that the cross-cluster merge costs more than the extra CTAs gain.
     // Up to 512 pages per (sequence, KV head) one cluster is faster (measured on the 8k stack).
     constexpr int per_cluster = DELTA_PAGES_PER_CLUSTER, one_cluster = DELTA_ONE_CLUSTER_PAGES;
-    const int max_clusters = (items <= one_cluster || items / per_cluster < 1) ? 1 : items / per_cluster;
+    const int max_clusters =
+        (one_cluster_per_unit || items <= one_cluster || items / per_cluster < 1) ? 1 : items / per_cluster;
     SplitPlan best = pl;
     int best_ctas = -1;
     for (int c = pl.cluster; c >= 1; --c) {
@@ -568,7 +572,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     int items = pt->max_pages_per_seq;
     if (mode == kModeSparse && sel_stride_in < items) items = sel_stride_in;
     const SplitPlan plan = fit_plan(plan_splits(d->dtype, D, pt->batch, Hkv, items), d->dtype, D, Hq / Hkv,
-                                    pt->batch * Hkv, items);
+                                    pt->batch * Hkv, items, mode == kModeDelta && !head_max);
     const int S = plan.splits();
     unsigned char* base = static_cast<unsigned char*>(ws);
 

@@ -66,20 +66,39 @@ struct SelectFinal {
 
 // Takes a ticket on `counter`; true in every thread of the CTA that arrives `expected`-th (which
 // also resets the counter for the next launch).  The CTA's earlier global writes are visible to
-// that CTA first.
+// that CTA first: the block barrier orders every thread's writes before thread 0's fence and
+// atomic, and the last CTA's thread 0 fences again before the barrier that releases its threads.
 __device__ __forceinline__ bool arrive_last(int* counter, int expected, uint32_t* s_flag) {
-    __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
+        __threadfence();
         const int t = atomicAdd(counter, 1);
         const uint32_t last = (t == expected - 1) ? 1u : 0u;
-        if (last) *counter = 0;
+        if (last) {
+            *counter = 0;
+            __threadfence();
+        }
         *s_flag = last;
     }
     __syncthreads();
-    const bool last = *s_flag != 0u;
-    if (last) __threadfence();
-    return last;
+    return *s_flag != 0u;
+}
+
+// Delta-layers, one cluster per unit: this CTA's page terms lse_hj for its first 2 NTHR pages,
+// loaded right after the loop (its warps wrote them before the preceding block barrier) so that
+// their latency overlaps the output merge.
+template <int NTHR, int G>
+__device__ __forceinline__ void select_preload(const DecodeParams& p, int b, int g, int N, float (&pre)[2][G]) {
+    const size_t maxp = size_t(p.max_pages);
+    const float* pl = p.page_lse + (size_t(b) * p.num_q_heads + g * G) * maxp;
+    const int i0 = blockIdx.x * p.items_per_split, i1 = min(i0 + p.items_per_split, N);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const int j = i0 + int(threadIdx.x) + i * NTHR;
+            pre[i][h] = (j < i1) ? pl[size_t(h) * maxp + j] : -INFINITY;
+        }
 }
 
 // Steps of the sequence's last CTA: page scores and their order keys, the threshold key T and the
@@ -98,8 +117,12 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     uint32_t* s_wmin = s_u + 8;                               // [W]
     uint32_t* s_wmax = s_wmin + W;                            // [W]
     constexpr size_t kScratch = ((256 + kTailList) * 4 + (W + 1) * 8 + 8 * 4 + 2 * W * 4 + 15) & ~size_t(15);
-    const int key_cap = int((free_bytes - kScratch) / 4);
-    uint32_t* keys = (N <= key_cap) ? reinterpret_cast<uint32_t*>(smem + kScratch) : a.keys + size_t(b) * maxp;
+    // keys in shared memory when they fit, one padding word after every 32 so that threads reading
+    // runs of consecutive pages hit different banks; else in the workspace
+    const int key_cap = int((free_bytes - kScratch) / 4 / 33 * 32);
+    const bool in_smem = N <= key_cap;
+    uint32_t* kbase = in_smem ? reinterpret_cast<uint32_t*>(smem + kScratch) : a.keys + size_t(b) * maxp;
+    auto KEY = [&](int j) -> uint32_t& { return kbase[in_smem ? j + (j >> 5) : j]; };
 
     // 1. page scores (the KV heads' shares summed in head order), order keys, candidate key range
     //    (candidates: pages neither sink nor recency)
@@ -110,15 +133,34 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     const bool radix = !take_all && k > 0;
     const float* us = a.unit_scores + size_t(b) * a.num_kv_heads * maxp;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int j = tid; j < N; j += NTHR) {
-        float sc = 0.f;
-        for (int u = 0; u < a.num_kv_heads; ++u) sc += __ldcg(us + size_t(u) * maxp + j);
-        if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
-        const uint32_t key = order_key(sc);
-        keys[j] = key;
-        if (j >= sinkP && j < recStart) {
-            kmin = min(kmin, key);
-            kmax = max(kmax, key);
+    // four pages per thread and eight KV heads at a time: 32 independent loads in flight
+    for (int jb = tid; jb < N; jb += 4 * NTHR) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int u0 = 0; u0 < a.num_kv_heads; u0 += 8) {
+            float v[8][4];
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int u = u0 + uu, j = jb + i * NTHR;
+                    v[uu][i] = (u < a.num_kv_heads && j < N) ? __ldcg(us + size_t(u) * maxp + j) : 0.f;
+                }
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] += v[uu][i];   // KV heads in order (adding 0 is exact)
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = jb + i * NTHR;
+            if (j >= N) break;
+            if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = acc[i];
+            const uint32_t key = order_key(acc[i]);
+            KEY(j) = key;
+            if (j >= sinkP && j < recStart) {
+                kmin = min(kmin, key);
+                kmax = max(kmax, key);
+            }
         }
     }
     kmin = __reduce_min_sync(0xffffffffu, kmin);
@@ -147,9 +189,17 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
             const int sh = max(0, 24 - __clz(span));   // (span >> sh) <= 255
             for (int i = tid; i < 256; i += NTHR) hist[i] = 0u;
             __syncthreads();
-            for (int j = sinkP + tid; j < recStart; j += NTHR) {
-                const uint32_t key = keys[j];
-                if (key >= lo && key - lo <= span) atomicAdd(&hist[(key - lo) >> sh], 1u);
+            // warp-aggregated: the many small scores crowd into a few buckets, so lanes with equal
+            // buckets add once (uniform trip count for the warp-wide match)
+            for (int base = sinkP; base < recStart; base += NTHR) {
+                const int j = base + tid;
+                uint32_t bin = 0xffffffffu;
+                if (j < recStart) {
+                    const uint32_t key = KEY(j);
+                    if (key >= lo && key - lo <= span) bin = (key - lo) >> sh;
+                }
+                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
             }
             __syncthreads();
             if (warp == 0) {   // lane covers buckets 255-8*lane .. 248-8*lane (descending)
@@ -203,7 +253,7 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
                 uint32_t key = 0;
                 bool in = false;
                 if (j < recStart) {
-                    key = keys[j];
+                    key = KEY(j);
                     in = key >= lo && key - lo <= span;
                 }
                 const uint32_t bal = __ballot_sync(0xffffffffu, in);
@@ -244,7 +294,7 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
         if (take_all || j < sinkP || j >= recStart) {
             ++take_cnt;
         } else if (radix) {
-            const uint32_t key = keys[j];
+            const uint32_t key = KEY(j);
             if (key > T) ++take_cnt;
             else if (key == T) ++eq_cnt;
         }
@@ -263,7 +313,7 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
         } else if (!radix) {
             take = false;
         } else {
-            const uint32_t key = keys[j];
+            const uint32_t key = KEY(j);
             take = key > T || (key == T && eq_seen++ < need);
         }
         if (take) {
@@ -279,7 +329,8 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
 // sequence's tokens and pages.
 template <int NTHR, int G, int D>
 __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char* smem, size_t free_bytes,
-                                            const float* recv, int b, int g, int n, int N) {
+                                            const float* recv, int b, int g, int n, int N,
+                                            const float (&pre)[2][G]) {
     constexpr int W = NTHR / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, S = p.num_splits, h0 = g * G;
@@ -288,15 +339,27 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
     uint32_t* s_flag = reinterpret_cast<uint32_t*>(s_c + kMaxGroup);
     const float* pl = p.page_lse + (size_t(b) * Hq + h0) * maxp;
     float* us = p.unit_scores + (size_t(b) * Hkv + g) * maxp;
-    // the unit's share of page j's score: the sum over its G heads of 2^(lse_hj - c_h)
-    auto share = [&](int j) {
-        float v[G];
+    // the unit's share of the scores of pages [j0, j1): the sum over its G heads of 2^(lse_hj - c_h),
+    // four pages per thread at a time (4 G independent loads in flight)
+    auto shares = [&](int j0, int j1) {
+        for (int jb = j0 + tid; jb < j1; jb += 4 * NTHR) {
+            float v[4][G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) v[h] = __ldcg(pl + size_t(h) * maxp + j);
-        float sc = 0.f;
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int h = 0; h < G; ++h) sc += exp2_approx(v[h] - s_c[h]);
-        return sc;
+                for (int h = 0; h < G; ++h) {
+                    const int j = jb + i * NTHR;
+                    v[i][h] = (j < j1) ? __ldcg(pl + size_t(h) * maxp + j) : -INFINITY;
+                }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = jb + i * NTHR;
+                float sc = 0.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h) sc += exp2_approx(v[i][h] - s_c[h]);
+                if (j < j1) us[j] = sc;
+            }
+        }
     };
     // c_h = log2 of the sum over states of l * 2^m (no token of the head: +inf, every term 0)
     auto norm = [](float M, float Z) { return (Z > 0.f) ? M + log2_approx(Z) : INFINITY; };
@@ -319,7 +382,15 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
         }
         __syncthreads();
         const int i0 = blockIdx.x * p.items_per_split, i1 = min(i0 + p.items_per_split, N);
-        for (int j = i0 + tid; j < i1; j += NTHR) us[j] = share(j);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {   // the preloaded pages
+            const int j = i0 + tid + i * NTHR;
+            float sc = 0.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h) sc += exp2_approx(pre[i][h] - s_c[h]);
+            if (j < i1) us[j] = sc;
+        }
+        shares(i0 + 2 * NTHR, i1);
         if (!arrive_last(p.seq_tickets + b, Hkv * S, s_flag)) return;
     } else {
         // the unit's last CTA forms c_h from the splits' states and writes the unit's shares
@@ -343,7 +414,7 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
             if (lane == 0) s_c[h] = norm(M, Z);
         }
         __syncthreads();
-        for (int j = tid; j < N; j += NTHR) us[j] = share(j);
+        shares(0, N);
         if (!arrive_last(p.seq_tickets + b, Hkv, s_flag)) return;
     }
     SelectFinal a;
