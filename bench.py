@@ -59,7 +59,44 @@ def parse(argv=None):
                     help="head aggregation of the page score: sum (default) or the page's max rule")
     ap.add_argument("--delta-sweep", type=str, default="",
                     help="comma list of delta-layer counts: time the step for each (spread placement)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="keep only the first N layers of the workload (same shapes; for profiler captures)")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="replay the decode step W + K times and exit without timing (for an ncu capture)")
     return ap.parse_args(argv)
+
+
+def workload(args):
+    """The selected workload, truncated to its first --layers layers when asked."""
+    from synth import configs as C
+    cfg = C.CONFIGS[args.config]
+    if args.layers and args.layers < cfg.num_layers:
+        dl = tuple(l for l in cfg.delta_layers if l < args.layers)
+        if not dl:
+            raise SystemExit("--layers must keep at least one delta-layer")
+        cfg = cfg.with_(name=f"{cfg.name}-first{args.layers}", num_layers=args.layers, delta_layers=dl)
+    return cfg
+
+
+def run_profile(args):
+    """Replay one decode step (the trajectory's first) W + K times: a short, fixed launch sequence for
+    a profiler (per step: the append, then one attention launch per layer)."""
+    import torch
+    from synth.case import Case
+    from synth.gpu import DeviceCase
+    cfg = workload(args)
+    if cfg.steps > 1:
+        cfg = cfg.with_(steps=1, drift_every=0)
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    case = Case(cfg)
+    dc = DeviceCase(case, device=device, prefill="append")
+    st = make_stacks(cfg, case, dc, args.reduce)(cfg.layer_kinds())
+    for _ in range(args.warmup + (args.steps or 3)):
+        st.step(dc.q, dc.k_new, dc.v_new, dc.k_pools, dc.v_pools, dc.out)
+    torch.cuda.synchronize()
+    print(f"profile run: {cfg.name}, {args.warmup + (args.steps or 3)} steps of {st.launches_per_step()} launches "
+          f"({', '.join(cfg.layer_kinds())})", flush=True)
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -532,35 +569,29 @@ def kernel_measurements(gpu, cfg, case, dc, d0, us_full_stack: float, k: int, wi
 
 
 def e2e_measure(gpu, cfg, dc, mk, k: int) -> dict:
-    """End to end through the public API with host buffers: every step the step's inputs (q, k_new,
-    v_new) go from one pinned host staging buffer to the device in one copy, the step runs (the
-    same C-ABI calls, captured in a graph over views of the device staging buffer) and every
-    layer's output comes back to pinned host memory."""
+    """End to end through the public API with host buffers (DeltaStack.step_host): every step the
+    appended tokens and every layer's q go from pinned host memory to the device (q layer by layer
+    on a copy stream, overlapping the earlier layers' attention), the step runs, and each layer's
+    output returns to pinned host memory as soon as its kernel is done; one CUDA graph per step."""
     import torch
-    nq, nk = dc.q.numel(), dc.k_new.numel()
-    in_h = torch.cat([dc.q.reshape(-1), dc.k_new.reshape(-1), dc.v_new.reshape(-1)]).cpu().pin_memory()
-    in_d = torch.empty_like(in_h, device=gpu.device)
-    in_d.copy_(in_h)
-    q_v = in_d[:nq].view_as(dc.q)
-    kn_v = in_d[nq:nq + nk].view_as(dc.k_new)
-    vn_v = in_d[nq + nk:].view_as(dc.v_new)
+    q_h, kn_h, vn_h = (x.cpu().pin_memory() for x in (dc.q, dc.k_new, dc.v_new))
     out_h = torch.empty_like(dc.out, device="cpu").pin_memory()
+    q_d, kn_d, vn_d = (torch.empty_like(x) for x in (dc.q, dc.k_new, dc.v_new))
     stack = mk(cfg.layer_kinds())
-    g = stack.capture(q_v, kn_v, vn_v, dc.k_pools, dc.v_pools, dc.out)
-
-    def step():
-        in_d.copy_(in_h, non_blocking=True)
-        g.replay()
-        out_h.copy_(dc.out, non_blocking=True)
-
-    us = gpu.mean_us(step, k)
-    e = in_h.element_size()
+    host_args = (q_h, kn_h, vn_h, dc.k_pools, dc.v_pools, out_h, q_d, kn_d, vn_d, dc.out)
+    stack.step_host(*host_args)   # outside capture: per-device kernel attributes, copy streams
+    torch.cuda.synchronize(gpu.device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        stack.step_host(*host_args)
+    us = gpu.mean_us(g.replay, k)
+    e = q_h.element_size()
     del g
-    stack.graph = None
-    return {"value": round(us, 3), "unit": UNIT, "h2d_bytes_per_step": in_h.numel() * e,
+    return {"value": round(us, 3), "unit": UNIT, "h2d_bytes_per_step": (q_h.numel() + kn_h.numel() + vn_h.numel()) * e,
             "d2h_bytes_per_step": out_h.numel() * e,
-            "how": "pinned host inputs -> device (one copy), graph replay of the step's C-ABI calls, every "
-                   "layer's output -> pinned host; CUDA events around the three"}
+            "how": "DeltaStack.step_host in one CUDA graph: pinned host k_new/v_new, then each layer's q, to the "
+                   "device on a copy stream; each layer's output to pinned host as its kernel ends; CUDA events "
+                   "around the replay"}
 
 
 def run_static(args, cfg, dist, rank, world, device, headline: bool = True) -> dict:
@@ -754,7 +785,7 @@ def run_ours(args):
     dist, rank, world, local = dist_init()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    cfg = C.CONFIGS[args.config]
+    cfg = workload(args)
     if cfg.steps > 1:
         r = run_trajectory(args, cfg, dist, rank, world, device)
         K = r["trajectory"]["timed_steps"]
@@ -842,9 +873,10 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    from synth import configs as C
-    if args.delta_sweep:
-        run_delta_sweep(args, C.CONFIGS[args.config], [int(x) for x in args.delta_sweep.split(",")])
+    if args.profile_run:
+        run_profile(args)
+    elif args.delta_sweep:
+        run_delta_sweep(args, workload(args), [int(x) for x in args.delta_sweep.split(",")])
     else:
         run_ours(args)
 

@@ -212,7 +212,8 @@ struct DecodeParams {
     int32_t* sel_pages_out;   // [B][sel_stride_out]
     int32_t sel_stride_out;
     float* page_scores;       // [B][max_pages] or null
-    float* unit_scores;       // [B][Hkv][max_pages] each (sequence, KV head) unit's share of the page scores
+    unsigned long long* score_acc;   // [B][max_pages] page scores in 2^-44 fixed point, summed over the
+                                     // KV heads by integer atomics; zero between launches
     uint32_t* keys;           // [B][max_pages] order keys of the page scores (when shared memory is short)
     int* unit_tickets;        // [B][Hkv] CTAs of a unit that finished, zero between launches
     int* seq_tickets;         // [B] units of a sequence that finished, zero between launches

@@ -55,7 +55,7 @@ enum : int { kVarNarrow = 0, kVarWide = 1, kVarShort = 2 };   // tensor-core ker
 constexpr int variant_threads(int v) { return 32 * (v == kVarWide ? kMmaWideWarps : v == kVarShort ? kMmaShortWarps : kWarps); }
 
 struct WsLayout {
-    size_t err, tickets, unit_tickets, seq_tickets, part_ml, part_o, page_lse, split_ml, unit_scores, keys, logits,
+    size_t err, tickets, unit_tickets, seq_tickets, part_ml, part_o, page_lse, split_ml, score_acc, keys, logits,
         total;
 };
 
@@ -218,7 +218,7 @@ WsLayout ws_layout(const delta_desc* d, int batch, int max_pages, bool with_logi
     w.part_o = off;       off += align256(rows * S * d->head_dim * sizeof(float));
     w.page_lse = off;     off += align256(rows * size_t(max_pages) * sizeof(float));
     w.split_ml = off;     off += align256(rows * S * sizeof(float2));
-    w.unit_scores = off;  off += align256(size_t(batch) * d->num_kv_heads * size_t(max_pages) * sizeof(float));
+    w.score_acc = off;    off += align256(size_t(batch) * size_t(max_pages) * sizeof(unsigned long long));
     w.keys = off;         off += align256(size_t(batch) * size_t(max_pages) * sizeof(uint32_t));
     w.logits = off;       off += with_logits ? align256(rows * size_t(max_pages) * kPage * sizeof(float)) : 0;
     w.total = off;
@@ -615,7 +615,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
         prm.sel_pages_out = sel_pages_out;
         prm.sel_stride_out = sel_stride_out;
         prm.page_scores = page_scores;
-        prm.unit_scores = reinterpret_cast<float*>(base + L.unit_scores);
+        prm.score_acc = reinterpret_cast<unsigned long long*>(base + L.score_acc);
         prm.keys = reinterpret_cast<uint32_t*>(base + L.keys);
         prm.unit_tickets = reinterpret_cast<int*>(base + L.unit_tickets);
         prm.seq_tickets = reinterpret_cast<int*>(base + L.seq_tickets);

@@ -9,65 +9,39 @@
 // (written by the decode loop) and c_h that head's log2-sum-exp over the whole context.
 //
 // No CTA waits for another.  When a (sequence, KV head) unit is one cluster, the output merge has
-// already given every CTA every split's state of the unit's heads, so each CTA forms c_h itself,
-// writes its own pages' share of the scores (the sum over the unit's G heads) and takes one
-// ticket on its sequence.  When a unit spans several clusters, each CTA takes a ticket on its
-// unit first, and the unit's last CTA forms c_h from the splits' states in the workspace and
-// writes the unit's shares.  The last CTA of the sequence sums the KV heads' shares (fixed order:
-// deterministic), finds the k-th largest candidate score by an adaptive-range radix select and
-// writes the ascending selection.
+// already given every CTA every split's state of the unit's heads, so each CTA forms c_h itself
+// and adds its own pages' share of the scores (the sum over the unit's G heads) into per-page
+// 2^-44 fixed-point accumulators with integer atomics (integer addition is associative, so the
+// sums do not depend on the order of arrival), then takes one ticket on its sequence.  When a
+// unit spans several clusters, each CTA takes a ticket on its unit first, and the unit's last CTA
+// forms c_h from the splits' states in the workspace and adds the unit's shares.  The last CTA of
+// the sequence reads the sums, finds the k-th largest candidate score by an adaptive-range radix
+// select and writes the ascending selection.
 #pragma once
 
 #include "common.cuh"
 
 namespace delta {
 
-constexpr int kTailList = 128;   // keys the final rank step compares pairwise, at most
-
-// Exclusive prefix sum of one 64-bit value per thread over a block of NTHR threads (a multiple
-// of 32, at most 1024).  `sums` holds NTHR/32 + 1 entries; it is not written again afterwards.
-template <int NTHR>
-__device__ __forceinline__ uint64_t block_scan_u64(uint64_t x, uint64_t* sums, uint64_t& total) {
-    constexpr int W = NTHR / 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint64_t incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const uint64_t w = lane < W ? sums[lane] : 0ull;
-        uint64_t wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint64_t y = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += y;
-        }
-        if (lane < W) sums[lane] = wi - w;   // exclusive prefix of the warp totals
-        if (lane == 31) sums[W] = wi;        // block total
-    }
-    __syncthreads();
-    total = sums[W];
-    return sums[warp] + incl - x;
-}
+constexpr int kTailList = 128;              // keys the final rank step compares pairwise, at most
+constexpr float kFixScale = 17592186044416.f;   // 2^44: fixed-point unit of the score accumulators
+constexpr float kFixInv = 5.684341886080802e-14f;   // 2^-44
 
 // What the sequence's last CTA needs (passed by value to the non-inlined final stage).
 struct SelectFinal {
-    const float* unit_scores;   // [B][Hkv][max_pages]
-    uint32_t* keys;             // [B][max_pages]
-    float* page_scores;         // [B][max_pages] or null
+    unsigned long long* score_acc;   // [B][max_pages]
+    uint32_t* keys;                  // [B][max_pages]
+    float* page_scores;              // [B][max_pages] or null
     int32_t* sel_cnt;
     int32_t* sel_pages;
-    int32_t sel_stride, max_pages, num_kv_heads, budget_pages, sink_tokens, recency_tokens;
+    int32_t sel_stride, max_pages, budget_pages, sink_tokens, recency_tokens;
 };
 
 // Takes a ticket on `counter`; true in every thread of the CTA that arrives `expected`-th (which
-// also resets the counter for the next launch).  The CTA's earlier global writes are visible to
-// that CTA first: the block barrier orders every thread's writes before thread 0's fence and
-// atomic, and the last CTA's thread 0 fences again before the barrier that releases its threads.
+// also resets the counter for the next launch).  The CTA's earlier global writes and reductions
+// are visible to that CTA first: the block barrier orders every thread's accesses before thread
+// 0's fence and atomic, and the last CTA's thread 0 fences again before the barrier that releases
+// its threads.
 __device__ __forceinline__ bool arrive_last(int* counter, int expected, uint32_t* s_flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -110,53 +84,42 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     constexpr int W = NTHR / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t maxp = size_t(a.max_pages);
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem);      // [256]
-    uint32_t* list = hist + 256;                              // [kTailList]
-    uint64_t* sums = reinterpret_cast<uint64_t*>(list + kTailList);   // [W + 1]
-    uint32_t* s_u = reinterpret_cast<uint32_t*>(sums + W + 1);        // [8] broadcasts
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem);      // [W][256] one histogram per warp
+    uint32_t* list = hist + W * 256;                          // [kTailList]
+    uint32_t* s_u = list + kTailList;                         // [8] broadcasts
     uint32_t* s_wmin = s_u + 8;                               // [W]
     uint32_t* s_wmax = s_wmin + W;                            // [W]
-    constexpr size_t kScratch = ((256 + kTailList) * 4 + (W + 1) * 8 + 8 * 4 + 2 * W * 4 + 15) & ~size_t(15);
-    // keys in shared memory when they fit, one padding word after every 32 so that threads reading
-    // runs of consecutive pages hit different banks; else in the workspace
-    const int key_cap = int((free_bytes - kScratch) / 4 / 33 * 32);
-    const bool in_smem = N <= key_cap;
-    uint32_t* kbase = in_smem ? reinterpret_cast<uint32_t*>(smem + kScratch) : a.keys + size_t(b) * maxp;
-    auto KEY = [&](int j) -> uint32_t& { return kbase[in_smem ? j + (j >> 5) : j]; };
+    uint32_t* s_wt = s_wmax + W;                              // [W] taken pages per warp segment
+    uint32_t* s_we = s_wt + W;                                // [W] pages equal to T per warp segment
+    constexpr size_t kScratch = ((W * 256 + kTailList + 8 + 4 * W) * 4 + 15) & ~size_t(15);
+    const int key_cap = int((free_bytes - kScratch) / 4);
+    uint32_t* keys = (N <= key_cap) ? reinterpret_cast<uint32_t*>(smem + kScratch) : a.keys + size_t(b) * maxp;
 
-    // 1. page scores (the KV heads' shares summed in head order), order keys, candidate key range
-    //    (candidates: pages neither sink nor recency)
+    // 1. page scores from the accumulators (which go back to zero for the next launch), order keys,
+    //    candidate key range (candidates: pages neither sink nor recency); eight loads in flight
     const int sinkP = min((min(a.sink_tokens, n) + kPage - 1) / kPage, N);
     const int recStart = (a.recency_tokens > 0) ? min(max(n - a.recency_tokens, 0) / kPage, N) : N;
     const int k = a.budget_pages;
     const bool take_all = max(recStart - sinkP, 0) <= k;
     const bool radix = !take_all && k > 0;
-    const float* us = a.unit_scores + size_t(b) * a.num_kv_heads * maxp;
+    unsigned long long* acc = a.score_acc + size_t(b) * maxp;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
-    // four pages per thread and eight KV heads at a time: 32 independent loads in flight
-    for (int jb = tid; jb < N; jb += 4 * NTHR) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int u0 = 0; u0 < a.num_kv_heads; u0 += 8) {
-            float v[8][4];
+    for (int jb = tid; jb < N; jb += 8 * NTHR) {
+        unsigned long long v[8];
 #pragma unroll
-            for (int uu = 0; uu < 8; ++uu)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int u = u0 + uu, j = jb + i * NTHR;
-                    v[uu][i] = (u < a.num_kv_heads && j < N) ? __ldcg(us + size_t(u) * maxp + j) : 0.f;
-                }
-#pragma unroll
-            for (int uu = 0; uu < 8; ++uu)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[i] += v[uu][i];   // KV heads in order (adding 0 is exact)
+        for (int i = 0; i < 8; ++i) {
+            const int j = jb + i * NTHR;
+            v[i] = (j < N) ? __ldcg(acc + j) : 0ull;
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
             const int j = jb + i * NTHR;
             if (j >= N) break;
-            if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = acc[i];
-            const uint32_t key = order_key(acc[i]);
-            KEY(j) = key;
+            acc[j] = 0ull;
+            const float sc = __ull2float_rn(v[i]) * kFixInv;
+            if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
+            const uint32_t key = order_key(sc);
+            keys[j] = key;
             if (j >= sinkP && j < recStart) {
                 kmin = min(kmin, key);
                 kmax = max(kmax, key);
@@ -187,19 +150,18 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
         bool exact = false;
         for (;;) {
             const int sh = max(0, 24 - __clz(span));   // (span >> sh) <= 255
-            for (int i = tid; i < 256; i += NTHR) hist[i] = 0u;
+            for (int i = tid; i < W * 256; i += NTHR) hist[i] = 0u;
             __syncthreads();
-            // warp-aggregated: the many small scores crowd into a few buckets, so lanes with equal
-            // buckets add once (uniform trip count for the warp-wide match)
-            for (int base = sinkP; base < recStart; base += NTHR) {
-                const int j = base + tid;
-                uint32_t bin = 0xffffffffu;
-                if (j < recStart) {
-                    const uint32_t key = KEY(j);
-                    if (key >= lo && key - lo <= span) bin = (key - lo) >> sh;
-                }
-                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
+            // per-warp histograms: same-bucket atomics contend only inside a warp
+            for (int j = sinkP + tid; j < recStart; j += NTHR) {
+                const uint32_t key = keys[j];
+                if (key >= lo && key - lo <= span) atomicAdd(&hist[warp * 256 + ((key - lo) >> sh)], 1u);
+            }
+            __syncthreads();
+            for (int i = tid; i < 256; i += NTHR) {
+                uint32_t c = 0;
+                for (int w = 0; w < W; ++w) c += hist[w * 256 + i];
+                hist[i] = c;   // warp 0's row becomes the total (each thread only reads its own column)
             }
             __syncthreads();
             if (warp == 0) {   // lane covers buckets 255-8*lane .. 248-8*lane (descending)
@@ -253,7 +215,7 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
                 uint32_t key = 0;
                 bool in = false;
                 if (j < recStart) {
-                    key = KEY(j);
+                    key = keys[j];
                     in = key >= lo && key - lo <= span;
                 }
                 const uint32_t bal = __ballot_sync(0xffffffffu, in);
@@ -284,49 +246,67 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
         }
     }
 
-    // 3. ascending compaction of sink U recency U {key > T} U {the first `need` keys == T}: each
-    //    thread owns a contiguous run of pages; one scan of the packed (equal, taken) counts gives
-    //    every thread its output position
-    const int per = (N + NTHR - 1) / NTHR;
-    const int jb = min(tid * per, N), je = min(jb + per, N);
-    uint32_t eq_cnt = 0, take_cnt = 0;
-    for (int j = jb; j < je; ++j) {
+    // 3. ascending compaction of sink U recency U {key > T} U {the first `need` keys == T}: warp w owns
+    //    a contiguous segment of pages and walks it 32 pages at a time (lane = page); ballots give the
+    //    ranks inside the warp, one exchange of the warps' totals gives the segments' offsets
+    const int seg = (((N + W - 1) / W) + 31) & ~31;
+    const int s0 = min(warp * seg, N), s1 = min(s0 + seg, N);
+    const uint32_t below = (1u << lane) - 1u;
+    auto classify = [&](int j, bool& tk, bool& eq) {
+        tk = false;
+        eq = false;
+        if (j >= s1) return;
         if (take_all || j < sinkP || j >= recStart) {
-            ++take_cnt;
+            tk = true;
         } else if (radix) {
-            const uint32_t key = KEY(j);
-            if (key > T) ++take_cnt;
-            else if (key == T) ++eq_cnt;
+            const uint32_t key = keys[j];
+            tk = key > T;
+            eq = key == T;
         }
+    };
+    uint32_t ct = 0, ce = 0;
+    for (int c = s0; c < s1; c += 32) {
+        bool tk, eq;
+        classify(c + lane, tk, eq);
+        ct += __popc(__ballot_sync(0xffffffffu, tk));
+        ce += __popc(__ballot_sync(0xffffffffu, eq));
     }
-    uint64_t tot;
-    const uint64_t pre = block_scan_u64<NTHR>(uint64_t(eq_cnt) | (uint64_t(take_cnt) << 32), sums, tot);
-    const uint32_t eq_rank = uint32_t(pre), take_rank = uint32_t(pre >> 32);
-    const uint32_t eq_tot = uint32_t(tot), take_tot = uint32_t(tot >> 32);
-    uint32_t pos = take_rank + min(need, eq_rank);
-    uint32_t eq_seen = eq_rank;
+    if (lane == 0) {
+        s_wt[warp] = ct;
+        s_we[warp] = ce;
+    }
+    __syncthreads();
+    uint32_t take_before = 0, eq_before = 0, take_tot = 0, eq_tot = 0;
+    for (int w = 0; w < W; ++w) {
+        if (w < warp) {
+            take_before += s_wt[w];
+            eq_before += s_we[w];
+        }
+        take_tot += s_wt[w];
+        eq_tot += s_we[w];
+    }
+    uint32_t pos = take_before + min(need, eq_before), eq_seen = eq_before;
     int32_t* out = a.sel_pages + size_t(b) * a.sel_stride;
-    for (int j = jb; j < je; ++j) {
-        bool take;
-        if (take_all || j < sinkP || j >= recStart) {
-            take = true;
-        } else if (!radix) {
-            take = false;
-        } else {
-            const uint32_t key = KEY(j);
-            take = key > T || (key == T && eq_seen++ < need);
-        }
+    for (int c = s0; c < s1; c += 32) {
+        const int j = c + lane;
+        bool tk, eq;
+        classify(j, tk, eq);
+        const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+        const bool take = tk || (eq && eq_seen + __popc(beq & below) < need);
+        const uint32_t bt = __ballot_sync(0xffffffffu, take);
         if (take) {
-            if (pos < uint32_t(a.sel_stride)) out[pos] = j;
-            ++pos;
+            const uint32_t at = pos + __popc(bt & below);
+            if (at < uint32_t(a.sel_stride)) out[at] = j;
         }
+        pos += __popc(bt);
+        eq_seen += __popc(beq);
     }
     if (tid == 0) a.sel_cnt[b] = int(min(take_tot + min(need, eq_tot), uint32_t(a.sel_stride)));
 }
 
 // Every thread of the CTA calls this after the output merge.  smem: the kernel's page-stage area,
 // idle by now (free_bytes long, 16-byte aligned); recv: the merge's receive area; n, N: the
-// sequence's tokens and pages.
+// sequence's tokens and pages; pre: select_preload's terms.
 template <int NTHR, int G, int D>
 __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char* smem, size_t free_bytes,
                                             const float* recv, int b, int g, int n, int N,
@@ -338,9 +318,15 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
     float* s_c = reinterpret_cast<float*>(smem);               // [kMaxGroup] per-head normalisers
     uint32_t* s_flag = reinterpret_cast<uint32_t*>(s_c + kMaxGroup);
     const float* pl = p.page_lse + (size_t(b) * Hq + h0) * maxp;
-    float* us = p.unit_scores + (size_t(b) * Hkv + g) * maxp;
-    // the unit's share of the scores of pages [j0, j1): the sum over its G heads of 2^(lse_hj - c_h),
-    // four pages per thread at a time (4 G independent loads in flight)
+    unsigned long long* acc = p.score_acc + size_t(b) * maxp;
+    // adds the unit's share of page j's score (the sum over its G heads of 2^(lse_hj - c_h))
+    auto add_share = [&](int j, const float (&v)[G]) {
+        float sc = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) sc += exp2_approx(v[h] - s_c[h]);
+        atomicAdd(acc + j, __float2ull_rn(sc * kFixScale));
+    };
+    // pages [j0, j1), four per thread at a time (4 G independent loads in flight)
     auto shares = [&](int j0, int j1) {
         for (int jb = j0 + tid; jb < j1; jb += 4 * NTHR) {
             float v[4][G];
@@ -352,13 +338,8 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
                     v[i][h] = (j < j1) ? __ldcg(pl + size_t(h) * maxp + j) : -INFINITY;
                 }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = jb + i * NTHR;
-                float sc = 0.f;
-#pragma unroll
-                for (int h = 0; h < G; ++h) sc += exp2_approx(v[i][h] - s_c[h]);
-                if (j < j1) us[j] = sc;
-            }
+            for (int i = 0; i < 4; ++i)
+                if (jb + i * NTHR < j1) add_share(jb + i * NTHR, v[i]);
         }
     };
     // c_h = log2 of the sum over states of l * 2^m (no token of the head: +inf, every term 0)
@@ -383,17 +364,12 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
         __syncthreads();
         const int i0 = blockIdx.x * p.items_per_split, i1 = min(i0 + p.items_per_split, N);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {   // the preloaded pages
-            const int j = i0 + tid + i * NTHR;
-            float sc = 0.f;
-#pragma unroll
-            for (int h = 0; h < G; ++h) sc += exp2_approx(pre[i][h] - s_c[h]);
-            if (j < i1) us[j] = sc;
-        }
+        for (int i = 0; i < 2; ++i)   // the preloaded pages
+            if (i0 + tid + i * NTHR < i1) add_share(i0 + tid + i * NTHR, pre[i]);
         shares(i0 + 2 * NTHR, i1);
         if (!arrive_last(p.seq_tickets + b, Hkv * S, s_flag)) return;
     } else {
-        // the unit's last CTA forms c_h from the splits' states and writes the unit's shares
+        // the unit's last CTA forms c_h from the splits' states and adds the unit's shares
         if (!arrive_last(p.unit_tickets + b * Hkv + g, S, s_flag)) return;
         for (int h = warp; h < G; h += W) {
             const float2* ps = p.split_ml + (size_t(b) * Hq + h0 + h) * S;
@@ -418,14 +394,13 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
         if (!arrive_last(p.seq_tickets + b, Hkv, s_flag)) return;
     }
     SelectFinal a;
-    a.unit_scores = p.unit_scores;
+    a.score_acc = p.score_acc;
     a.keys = p.keys;
     a.page_scores = p.page_scores;
     a.sel_cnt = p.sel_cnt_out;
     a.sel_pages = p.sel_pages_out;
     a.sel_stride = p.sel_stride_out;
     a.max_pages = p.max_pages;
-    a.num_kv_heads = Hkv;
     a.budget_pages = p.budget_pages;
     a.sink_tokens = p.sink_tokens;
     a.recency_tokens = p.recency_tokens;

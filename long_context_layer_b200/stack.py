@@ -75,26 +75,82 @@ class DeltaStack:
 
     def step(self, q, k_new, v_new, k_pools, v_pools, out, append: bool = True, stream: int | None = None):
         st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
-        d, pt, ws, wb = self.desc, self.pt, self.workspace, self.ws_bytes
+        d, pt = self.desc, self.pt
         cur = -1
         if append:      # every layer's new token in one launch (layers do not read each other's pools)
             N.kv_append_layers(d, pt, k_new, v_new, k_pools, v_pools, st)
         for l, kind in enumerate(self.kinds):
-            if kind == FULL:
-                N.full_attn(d, pt, q[l], k_pools[l], v_pools[l], out[l], ws, wb, st)
-            elif kind == DELTA:
+            # a sparse layer after a sparse layer uses the settled entry: the selection and the
+            # appended tokens were final before the previous sparse layer began (it waited on the
+            # delta-layer that wrote the selection), so this layer may read them early
+            self._layer(l, kind, cur, q, k_pools, v_pools, out, st)
+            if kind == DELTA:
                 cur = self.delta_layers.index(l)
-                scores = self.page_scores[cur] if self.page_scores is not None else None
-                N.select_attn(d, pt, self.sp, q[l], k_pools[l], v_pools[l], out[l], self.sel_cnt[cur],
-                              self.sel_pages[cur], self.sel_stride, scores, ws, wb, st)
-            elif l > 0 and self.kinds[l - 1] == SPARSE:
-                # the selection and the appended tokens were final before the previous sparse layer
-                # began (it waited on the selection kernel), so this layer may read them early
-                N.sparse_attn_settled(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l],
-                                      k_pools[l], v_pools[l], out[l], ws, wb, st)
-            else:
-                N.sparse_attn(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l], k_pools[l],
-                              v_pools[l], out[l], ws, wb, st)
+
+    # ------------------------------------------------------------------ host buffers
+    def step_host(self, q_host, k_new_host, v_new_host, k_pools, v_pools, out_host, q_dev, k_new_dev, v_new_dev,
+                  out_dev, append: bool = True):
+        """One decode step whose inputs and outputs live in (pinned) host memory.
+
+        The appended tokens go to the device first (every layer's append needs them), then each
+        layer's q on a copy stream while the earlier layers compute; each layer's output returns to
+        the host on another stream as soon as its kernel is done.  *_dev are device staging buffers
+        of the same shapes.  Every call is enqueued on the current stream (graph-capturable);
+        out_host is complete once that stream reaches the end of the step.
+        """
+        main = torch.cuda.current_stream(self.device)
+        if not hasattr(self, "_up"):
+            self._up = torch.cuda.Stream(self.device)
+            self._down = torch.cuda.Stream(self.device)
+        up, down = self._up, self._down
+        L = len(self.kinds)
+        up.wait_stream(main)
+        down.wait_stream(main)
+        with torch.cuda.stream(up):
+            k_new_dev.copy_(k_new_host, non_blocking=True)
+            v_new_dev.copy_(v_new_host, non_blocking=True)
+            kv_ready = torch.cuda.Event()
+            kv_ready.record(up)
+            q_ready = []
+            for l in range(L):
+                q_dev[l].copy_(q_host[l], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(up)
+                q_ready.append(ev)
+        main.wait_event(kv_ready)
+        st = main.cuda_stream
+        d, pt, ws, wb = self.desc, self.pt, self.workspace, self.ws_bytes
+        if append:
+            N.kv_append_layers(d, pt, k_new_dev, v_new_dev, k_pools, v_pools, st)
+        cur = -1
+        for l, kind in enumerate(self.kinds):
+            main.wait_event(q_ready[l])
+            self._layer(l, kind, cur, q_dev, k_pools, v_pools, out_dev, st)
+            if kind == DELTA:
+                cur = self.delta_layers.index(l)
+            done = torch.cuda.Event()
+            done.record(main)
+            down.wait_event(done)
+            with torch.cuda.stream(down):
+                out_host[l].copy_(out_dev[l], non_blocking=True)
+        main.wait_stream(up)
+        main.wait_stream(down)
+
+    def _layer(self, l, kind, cur, q, k_pools, v_pools, out, st):
+        d, pt, ws, wb = self.desc, self.pt, self.workspace, self.ws_bytes
+        if kind == FULL:
+            N.full_attn(d, pt, q[l], k_pools[l], v_pools[l], out[l], ws, wb, st)
+        elif kind == DELTA:
+            c = self.delta_layers.index(l)
+            scores = self.page_scores[c] if self.page_scores is not None else None
+            N.select_attn(d, pt, self.sp, q[l], k_pools[l], v_pools[l], out[l], self.sel_cnt[c], self.sel_pages[c],
+                          self.sel_stride, scores, ws, wb, st)
+        elif l > 0 and self.kinds[l - 1] == SPARSE:
+            N.sparse_attn_settled(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l], k_pools[l],
+                                  v_pools[l], out[l], ws, wb, st)
+        else:
+            N.sparse_attn(d, pt, self.sel_cnt[cur], self.sel_pages[cur], self.sel_stride, q[l], k_pools[l],
+                          v_pools[l], out[l], ws, wb, st)
 
     # ------------------------------------------------------------------ CUDA graph
     def capture(self, *args, **kw) -> torch.cuda.CUDAGraph:

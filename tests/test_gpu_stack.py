@@ -111,3 +111,30 @@ def test_full_size_workload_sampled(cfg, layers, batch):
     run(stack, dc)
     # every delta-layer's selection is checked for the sampled sequences, outputs of the sampled layers
     check_stack_against_oracle(cfg, case, dc, stack, layers=layers, batch=batch)
+
+
+@pytest.mark.parametrize("cfg", [C.TINY, C.QWEN7B_8K])
+def test_step_host_matches_the_device_step(cfg):
+    # the host-buffer step (per-layer uploads and downloads on copy streams) runs the same kernels on
+    # the same values: the same bits as the device-buffer step, eagerly and replayed from a graph
+    case, dc, stack = build(cfg)
+    run(stack, dc)
+    ref = dc.out.clone()
+    ref_sel = stack.sel_pages.clone()
+    q_h, kn_h, vn_h = (x.cpu().pin_memory() for x in (dc.q, dc.k_new, dc.v_new))
+    out_h = torch.full(tuple(dc.out.shape), float("nan"), dtype=dc.out.dtype).pin_memory()
+    q_d, kn_d, vn_d = (torch.zeros_like(x) for x in (dc.q, dc.k_new, dc.v_new))
+    args = (q_h, kn_h, vn_h, dc.k_pools, dc.v_pools, out_h, q_d, kn_d, vn_d, dc.out)
+    dc.out.zero_()
+    stack.step_host(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, ref.cpu())
+    assert torch.equal(stack.sel_pages, ref_sel)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        stack.step_host(*args)
+    for _ in range(3):
+        out_h.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out_h, ref.cpu())
