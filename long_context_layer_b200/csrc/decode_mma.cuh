@@ -242,9 +242,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
     auto parity = [&](int k) -> uint32_t { return ((k / STAGES) + ((spec_used >> (k % STAGES)) & 1u)) & 1u; };
 
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2*t4, 2*t4+1
-    // delta-layers: the same state over the pages' fp32 terms (l_run sums the bf16-rounded
-    // probabilities that also weight V), so the selection's normalisers match its page terms
-    float dm_run[2] = {-INFINITY, -INFINITY}, dl_run[2] = {0.f, 0.f};
+    // delta-layers: the sum of the unrounded fp32 terms 2^(s - m_run) (l_run sums the bf16-rounded
+    // probabilities that also weight V), so the selection's normalisers match its page terms; its
+    // maximum is m_run
+    float dl_run[2] = {0.f, 0.f};
     float acc[KS][4];
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
@@ -279,36 +280,37 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
         sc[2] = ok1 ? (c0[2] + c1[2]) * p.qscale : -INFINITY;
         sc[3] = ok1 ? (c0[3] + c1[3]) * p.qscale : -INFINITY;
     };
-    // Delta-layers: page partials from the unrounded probabilities (max logit, sum of 2^(s - max))
-    auto page_partials = [&](const float (&sc)[4], int lp) {
-        if (p.logits != nullptr) {
-            // per-token logits of this page (HEAD_MAX scoring): tokens g4, g4+8; heads 2*t4, 2*t4+1
-            float* lg = p.logits + (size_t(b) * Hq + h0) * (size_t(p.max_pages) * kPage) + size_t(lp) * kPage;
-            const size_t hs = size_t(p.max_pages) * kPage;
-            if (2 * t4 < G) { lg[2 * t4 * hs + g4] = sc[0]; lg[2 * t4 * hs + g4 + 8] = sc[2]; }
-            if (2 * t4 + 1 < G) { lg[(2 * t4 + 1) * hs + g4] = sc[1]; lg[(2 * t4 + 1) * hs + g4 + 8] = sc[3]; }
-        }
-        float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+    // Delta-layers: each page's log2-sum-exp per head, from the same unrounded terms 2^(s - m) the
+    // online softmax forms (m: the running maximum over both pages), summed over the page's 16
+    // tokens (the g4 lanes), and the fp32-term running sum.  p*: a lane's terms of page A / B
+    // (tokens g4, g4 + 8; heads 2 t4, 2 t4 + 1); al: the softmax's rescale factors.
+    auto page_partials = [&](const float (&pa)[4], const float (&pb)[4], float mn0, float mn1, float al0, float al1,
+                             bool vA, bool vB, int lpA, int lpB) {
+        float ea0 = pa[0] + pa[2], ea1 = pa[1] + pa[3], eb0 = pb[0] + pb[2], eb1 = pb[1] + pb[3];
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+            ea0 += __shfl_xor_sync(0xffffffffu, ea0, o);
+            ea1 += __shfl_xor_sync(0xffffffffu, ea1, o);
+            eb0 += __shfl_xor_sync(0xffffffffu, eb0, o);
+            eb1 += __shfl_xor_sync(0xffffffffu, eb1, o);
         }
-        float e0 = exp2_approx(sc[0] - mx0) + exp2_approx(sc[2] - mx0);
-        float e1 = exp2_approx(sc[1] - mx1) + exp2_approx(sc[3] - mx1);
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-            e0 += __shfl_xor_sync(0xffffffffu, e0, o);
-            e1 += __shfl_xor_sync(0xffffffffu, e1, o);
-        }
-        const float n0 = fmaxf(dm_run[0], mx0), n1 = fmaxf(dm_run[1], mx1);   // finite: the page is valid
-        dl_run[0] = dl_run[0] * exp2_approx(dm_run[0] - n0) + e0 * exp2_approx(mx0 - n0);
-        dl_run[1] = dl_run[1] * exp2_approx(dm_run[1] - n1) + e1 * exp2_approx(mx1 - n1);
-        dm_run[0] = n0;
-        dm_run[1] = n1;
+        dl_run[0] = dl_run[0] * al0 + (ea0 + eb0);
+        dl_run[1] = dl_run[1] * al1 + (ea1 + eb1);
         const int hA = 2 * t4, hB = 2 * t4 + 1;
-        if (g4 == 0 && hA < G) p.page_lse[(size_t(b) * Hq + h0 + hA) * p.max_pages + lp] = mx0 + log2_approx(e0);
-        if (g4 == 0 && hB < G) p.page_lse[(size_t(b) * Hq + h0 + hB) * p.max_pages + lp] = mx1 + log2_approx(e1);
+        if (g4 == 0) {
+            float* row = p.page_lse + (size_t(b) * Hq + h0) * p.max_pages;
+            if (vA && hA < G) row[size_t(hA) * p.max_pages + lpA] = mn0 + log2_approx(ea0);
+            if (vA && hB < G) row[size_t(hB) * p.max_pages + lpA] = mn1 + log2_approx(ea1);
+            if (vB && hA < G) row[size_t(hA) * p.max_pages + lpB] = mn0 + log2_approx(eb0);
+            if (vB && hB < G) row[size_t(hB) * p.max_pages + lpB] = mn1 + log2_approx(eb1);
+        }
+    };
+    // HEAD_MAX scoring: every head's per-token logits (tokens g4, g4 + 8; heads 2 t4, 2 t4 + 1)
+    auto store_logits = [&](const float (&sc)[4], int lp) {
+        float* lg = p.logits + (size_t(b) * Hq + h0) * (size_t(p.max_pages) * kPage) + size_t(lp) * kPage;
+        const size_t hs = size_t(p.max_pages) * kPage;
+        if (2 * t4 < G) { lg[2 * t4 * hs + g4] = sc[0]; lg[2 * t4 * hs + g4 + 8] = sc[2]; }
+        if (2 * t4 + 1 < G) { lg[(2 * t4 + 1) * hs + g4] = sc[1]; lg[(2 * t4 + 1) * hs + g4 + 8] = sc[3]; }
     };
     // tokens past the end of the context: zero their V rows (they may hold non-finite bytes)
     auto zero_tail = [&](int s, int tv) {
@@ -357,9 +359,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
         if (vB) qk_page(sB, tvB, scB);
         bool zeroed = false;
         if (vA || vB) {
-            if (p.mode == kModeDelta) {
-                if (vA) page_partials(scA, lpA);
-                if (vB) page_partials(scB, lpB);
+            if (p.logits != nullptr) {
+                if (vA) store_logits(scA, lpA);
+                if (vB) store_logits(scB, lpB);
             }
             float mx0 = fmaxf(fmaxf(scA[0], scA[2]), fmaxf(scB[0], scB[2]));
             float mx1 = fmaxf(fmaxf(scA[1], scA[3]), fmaxf(scB[1], scB[3]));
@@ -370,10 +372,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
             }
             const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);   // finite: a valid token exists
             const float al0 = exp2_approx(m_run[0] - mn0), al1 = exp2_approx(m_run[1] - mn1);
-            const uint32_t xa0 = pack_bf16(exp2_approx(scA[0] - mn0), exp2_approx(scA[1] - mn1));
-            const uint32_t xa1 = pack_bf16(exp2_approx(scA[2] - mn0), exp2_approx(scA[3] - mn1));
-            const uint32_t xb0 = pack_bf16(exp2_approx(scB[0] - mn0), exp2_approx(scB[1] - mn1));
-            const uint32_t xb1 = pack_bf16(exp2_approx(scB[2] - mn0), exp2_approx(scB[3] - mn1));
+            const float pa[4] = {exp2_approx(scA[0] - mn0), exp2_approx(scA[1] - mn1), exp2_approx(scA[2] - mn0),
+                                 exp2_approx(scA[3] - mn1)};
+            const float pb[4] = {exp2_approx(scB[0] - mn0), exp2_approx(scB[1] - mn1), exp2_approx(scB[2] - mn0),
+                                 exp2_approx(scB[3] - mn1)};
+            if (p.mode == kModeDelta) page_partials(pa, pb, mn0, mn1, al0, al1, vA, vB, lpA, lpB);
+            const uint32_t xa0 = pack_bf16(pa[0], pa[1]);
+            const uint32_t xa1 = pack_bf16(pa[2], pa[3]);
+            const uint32_t xb0 = pack_bf16(pb[0], pb[1]);
+            const uint32_t xb1 = pack_bf16(pb[2], pb[3]);
             float p0, p1, p2, p3, q0, q1, q2, q3;
             unpack_bf16x2(xa0, p0, p1);
             unpack_bf16x2(xa1, p2, p3);
@@ -433,9 +440,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
         pml[(2 * t4 + 1) * 2 + 0] = m_run[1];
         pml[(2 * t4 + 1) * 2 + 1] = l_run[1];
         if (p.mode == kModeDelta) {
-            pdl[(2 * t4) * 2 + 0] = dm_run[0];
+            pdl[(2 * t4) * 2 + 0] = m_run[0];
             pdl[(2 * t4) * 2 + 1] = dl_run[0];
-            pdl[(2 * t4 + 1) * 2 + 0] = dm_run[1];
+            pdl[(2 * t4 + 1) * 2 + 0] = m_run[1];
             pdl[(2 * t4 + 1) * 2 + 1] = dl_run[1];
         }
     }

@@ -89,14 +89,17 @@ class DeltaStack:
 
     # ------------------------------------------------------------------ host buffers
     def step_host(self, q_host, k_new_host, v_new_host, k_pools, v_pools, out_host, q_dev, k_new_dev, v_new_dev,
-                  out_dev, append: bool = True):
+                  out_dev, append: bool = True, early_layers: int = 2, out_chunks: int = 8):
         """One decode step whose inputs and outputs live in (pinned) host memory.
 
-        The appended tokens go to the device first (every layer's append needs them), then each
-        layer's q on a copy stream while the earlier layers compute; each layer's output returns to
-        the host on another stream as soon as its kernel is done.  *_dev are device staging buffers
-        of the same shapes.  Every call is enqueued on the current stream (graph-capturable);
-        out_host is complete once that stream reaches the end of the step.
+        On a copy stream: the first `early_layers` layers' q and the appended tokens (every
+        layer's append needs them), then the other layers' q, which arrive while the first
+        layers compute.  The outputs return to the host on another stream in `out_chunks`
+        groups of consecutive layers, each as soon as its last layer is done.  The compute
+        stream joins the copy streams at those few points only, so most consecutive kernels keep
+        their programmatic-launch overlap.  *_dev are device staging buffers of the same shapes.
+        Everything is enqueued on the current stream (graph-capturable); out_host is complete
+        once that stream reaches the end of the step.
         """
         main = torch.cuda.current_stream(self.device)
         if not hasattr(self, "_up"):
@@ -104,35 +107,39 @@ class DeltaStack:
             self._down = torch.cuda.Stream(self.device)
         up, down = self._up, self._down
         L = len(self.kinds)
+        early = max(1, min(early_layers, L))
         up.wait_stream(main)
         down.wait_stream(main)
         with torch.cuda.stream(up):
+            q_dev[:early].copy_(q_host[:early], non_blocking=True)
             k_new_dev.copy_(k_new_host, non_blocking=True)
             v_new_dev.copy_(v_new_host, non_blocking=True)
-            kv_ready = torch.cuda.Event()
-            kv_ready.record(up)
-            q_ready = []
-            for l in range(L):
-                q_dev[l].copy_(q_host[l], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(up)
-                q_ready.append(ev)
-        main.wait_event(kv_ready)
+            first_ready = torch.cuda.Event()
+            first_ready.record(up)
+            rest_ready = None
+            if early < L:
+                q_dev[early:].copy_(q_host[early:], non_blocking=True)
+                rest_ready = torch.cuda.Event()
+                rest_ready.record(up)
+        main.wait_event(first_ready)
         st = main.cuda_stream
-        d, pt, ws, wb = self.desc, self.pt, self.workspace, self.ws_bytes
         if append:
-            N.kv_append_layers(d, pt, k_new_dev, v_new_dev, k_pools, v_pools, st)
-        cur = -1
+            N.kv_append_layers(self.desc, self.pt, k_new_dev, v_new_dev, k_pools, v_pools, st)
+        per = -(-L // max(1, out_chunks))
+        cur, c0 = -1, 0
         for l, kind in enumerate(self.kinds):
-            main.wait_event(q_ready[l])
+            if l == early and rest_ready is not None:
+                main.wait_event(rest_ready)
             self._layer(l, kind, cur, q_dev, k_pools, v_pools, out_dev, st)
             if kind == DELTA:
                 cur = self.delta_layers.index(l)
-            done = torch.cuda.Event()
-            done.record(main)
-            down.wait_event(done)
-            with torch.cuda.stream(down):
-                out_host[l].copy_(out_dev[l], non_blocking=True)
+            if l + 1 - c0 == per or l == L - 1:
+                done = torch.cuda.Event()
+                done.record(main)
+                down.wait_event(done)
+                with torch.cuda.stream(down):
+                    out_host[c0:l + 1].copy_(out_dev[c0:l + 1], non_blocking=True)
+                c0 = l + 1
         main.wait_stream(up)
         main.wait_stream(down)
 
