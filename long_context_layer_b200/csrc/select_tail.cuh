@@ -96,7 +96,7 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     uint32_t* keys = (N <= key_cap) ? reinterpret_cast<uint32_t*>(smem + kScratch) : a.keys + size_t(b) * maxp;
 
     // 1. page scores from the accumulators (which go back to zero for the next launch), order keys,
-    //    candidate key range (candidates: pages neither sink nor recency); eight loads in flight
+    //    candidate key range (candidates: pages neither sink nor recency); sixteen loads in flight
     const int sinkP = min((min(a.sink_tokens, n) + kPage - 1) / kPage, N);
     const int recStart = (a.recency_tokens > 0) ? min(max(n - a.recency_tokens, 0) / kPage, N) : N;
     const int k = a.budget_pages;
@@ -104,15 +104,15 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     const bool radix = !take_all && k > 0;
     unsigned long long* acc = a.score_acc + size_t(b) * maxp;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int jb = tid; jb < N; jb += 8 * NTHR) {
-        unsigned long long v[8];
+    for (int jb = tid; jb < N; jb += 16 * NTHR) {
+        unsigned long long v[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 16; ++i) {
             const int j = jb + i * NTHR;
             v[i] = (j < N) ? __ldcg(acc + j) : 0ull;
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 16; ++i) {
             const int j = jb + i * NTHR;
             if (j >= N) break;
             acc[j] = 0ull;
@@ -152,10 +152,19 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
             const int sh = max(0, 24 - __clz(span));   // (span >> sh) <= 255
             for (int i = tid; i < W * 256; i += NTHR) hist[i] = 0u;
             __syncthreads();
-            // per-warp histograms: same-bucket atomics contend only inside a warp
-            for (int j = sinkP + tid; j < recStart; j += NTHR) {
-                const uint32_t key = keys[j];
-                if (key >= lo && key - lo <= span) atomicAdd(&hist[warp * 256 + ((key - lo) >> sh)], 1u);
+            // per-warp histograms: same-bucket atomics contend only inside a warp; eight keys per thread
+            // are loaded before their atomics so the loads overlap
+            for (int j0 = sinkP + tid; j0 < recStart; j0 += 8 * NTHR) {
+                uint32_t kv[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int j = j0 + i * NTHR;
+                    kv[i] = (j < recStart) ? keys[j] : 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (j0 + i * NTHR < recStart && kv[i] >= lo && kv[i] - lo <= span)
+                        atomicAdd(&hist[warp * 256 + ((kv[i] - lo) >> sh)], 1u);
             }
             __syncthreads();
             for (int i = tid; i < 256; i += NTHR) {
@@ -264,12 +273,17 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
             eq = key == T;
         }
     };
+    // four groups of 32 pages per step: their key loads and ballots are independent
     uint32_t ct = 0, ce = 0;
-    for (int c = s0; c < s1; c += 32) {
-        bool tk, eq;
-        classify(c + lane, tk, eq);
-        ct += __popc(__ballot_sync(0xffffffffu, tk));
-        ce += __popc(__ballot_sync(0xffffffffu, eq));
+    for (int c = s0; c < s1; c += 128) {
+        bool tk[4], eq[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) classify(c + 32 * u + lane, tk[u], eq[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            ct += __popc(__ballot_sync(0xffffffffu, tk[u]));
+            ce += __popc(__ballot_sync(0xffffffffu, eq[u]));
+        }
     }
     if (lane == 0) {
         s_wt[warp] = ct;
@@ -287,19 +301,24 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     }
     uint32_t pos = take_before + min(need, eq_before), eq_seen = eq_before;
     int32_t* out = a.sel_pages + size_t(b) * a.sel_stride;
-    for (int c = s0; c < s1; c += 32) {
-        const int j = c + lane;
-        bool tk, eq;
-        classify(j, tk, eq);
-        const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-        const bool take = tk || (eq && eq_seen + __popc(beq & below) < need);
-        const uint32_t bt = __ballot_sync(0xffffffffu, take);
-        if (take) {
-            const uint32_t at = pos + __popc(bt & below);
-            if (at < uint32_t(a.sel_stride)) out[at] = j;
+    for (int c = s0; c < s1; c += 128) {
+        bool tk[4], eq[4];
+        uint32_t beq[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) classify(c + 32 * u + lane, tk[u], eq[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) beq[u] = __ballot_sync(0xffffffffu, eq[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {   // in page order: the ranks carry from group to group
+            const bool take = tk[u] || (eq[u] && eq_seen + __popc(beq[u] & below) < need);
+            const uint32_t bt = __ballot_sync(0xffffffffu, take);
+            if (take) {
+                const uint32_t at = pos + __popc(bt & below);
+                if (at < uint32_t(a.sel_stride)) out[at] = c + 32 * u + lane;
+            }
+            pos += __popc(bt);
+            eq_seen += __popc(beq[u]);
         }
-        pos += __popc(bt);
-        eq_seen += __popc(beq);
     }
     if (tid == 0) a.sel_cnt[b] = int(min(take_tot + min(need, eq_tot), uint32_t(a.sel_stride)));
 }
