@@ -114,15 +114,15 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int j = jb + i * NTHR;
-            if (j >= N) break;
-            acc[j] = 0ull;
             const float sc = __ull2float_rn(v[i]) * kFixInv;
-            if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
             const uint32_t key = order_key(sc);
-            keys[j] = key;
-            if (j >= sinkP && j < recStart) {
-                kmin = min(kmin, key);
-                kmax = max(kmax, key);
+            const bool cand = (j >= sinkP) & (j < recStart);   // (implies j < N)
+            kmin = cand ? min(kmin, key) : kmin;
+            kmax = cand ? max(kmax, key) : kmax;
+            if (j < N) {
+                acc[j] = 0ull;
+                keys[j] = key;
+                if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
             }
         }
     }
@@ -219,19 +219,30 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
             // gather the bucket's keys (at most kTailList) and rank them exactly
             if (tid == 0) s_u[4] = 0;
             __syncthreads();
-            for (int base = sinkP; base < recStart; base += NTHR) {   // uniform trip count for the ballot
-                const int j = base + tid;
-                uint32_t key = 0;
-                bool in = false;
-                if (j < recStart) {
-                    key = keys[j];
-                    in = key >= lo && key - lo <= span;
+            // four groups of NTHR keys per step (uniform trip count for the ballots): loads first, then
+            // one slot reservation per warp for all four groups
+            for (int base = sinkP; base < recStart; base += 4 * NTHR) {
+                uint32_t kv[4], bal[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = base + u * NTHR + tid;
+                    kv[u] = (j < recStart) ? keys[j] : 0u;
                 }
-                const uint32_t bal = __ballot_sync(0xffffffffu, in);
+                uint32_t cnt = 0;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = base + u * NTHR + tid;
+                    bal[u] = __ballot_sync(0xffffffffu, (j < recStart) & (kv[u] >= lo) & (kv[u] - lo <= span));
+                    cnt += __popc(bal[u]);
+                }
                 uint32_t slot = 0;
-                if (lane == 0 && bal != 0u) slot = atomicAdd(&s_u[4], uint32_t(__popc(bal)));
+                if (lane == 0 && cnt != 0u) slot = atomicAdd(&s_u[4], cnt);
                 slot = __shfl_sync(0xffffffffu, slot, 0);
-                if (in) list[slot + __popc(bal & ((1u << lane) - 1u))] = key;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if ((bal[u] >> lane) & 1u) list[slot + __popc(bal[u] & ((1u << lane) - 1u))] = kv[u];
+                    slot += __popc(bal[u]);
+                }
             }
             __syncthreads();
             const int m = int(s_u[4]);
@@ -261,24 +272,28 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     const int seg = (((N + W - 1) / W) + 31) & ~31;
     const int s0 = min(warp * seg, N), s1 = min(s0 + seg, N);
     const uint32_t below = (1u << lane) - 1u;
-    auto classify = [&](int j, bool& tk, bool& eq) {
-        tk = false;
-        eq = false;
-        if (j >= s1) return;
-        if (take_all || j < sinkP || j >= recStart) {
-            tk = true;
-        } else if (radix) {
-            const uint32_t key = keys[j];
-            tk = key > T;
-            eq = key == T;
+    // four groups of 32 pages per step, branch-free: the key loads first, then the flags (a page is
+    // taken if forced or above T; equal to T is decided by rank)
+    auto classify4 = [&](int c, bool (&tk)[4], bool (&eq)[4]) {
+        uint32_t kv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = c + 32 * u + lane;
+            kv[u] = (j < s1) ? keys[j] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = c + 32 * u + lane;
+            const bool inr = j < s1;
+            const bool forced = take_all | (j < sinkP) | (j >= recStart);
+            tk[u] = inr & (forced | (radix & (kv[u] > T)));
+            eq[u] = inr & !forced & radix & (kv[u] == T);
         }
     };
-    // four groups of 32 pages per step: their key loads and ballots are independent
     uint32_t ct = 0, ce = 0;
     for (int c = s0; c < s1; c += 128) {
         bool tk[4], eq[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) classify(c + 32 * u + lane, tk[u], eq[u]);
+        classify4(c, tk, eq);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             ct += __popc(__ballot_sync(0xffffffffu, tk[u]));
@@ -304,8 +319,7 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
     for (int c = s0; c < s1; c += 128) {
         bool tk[4], eq[4];
         uint32_t beq[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) classify(c + 32 * u + lane, tk[u], eq[u]);
+        classify4(c, tk, eq);
 #pragma unroll
         for (int u = 0; u < 4; ++u) beq[u] = __ballot_sync(0xffffffffu, eq[u]);
 #pragma unroll
