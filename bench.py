@@ -711,7 +711,7 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
             events.append((s0, s1))
         else:
             g.replay()
-        if step in checks:
+        if step in checks:   # copies only: the oracle runs after the timed loop (host cores stay free)
             cnt = stack.sel_cnt.cpu().numpy()
             pages = stack.sel_pages.cpu().numpy()
             outs = dc.out[ld].float().cpu().numpy()
@@ -719,9 +719,11 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
                 for b in range(cfg.batch):
                     gpu_sel[(step, l, b)] = pages[i, b, :cnt[i, b]].tolist()
                     gpu_out[(step, l, b)] = outs[i, b]
-            pending.append(pool.submit([(cfg, step, "delta", l, b) for l in ld for b in range(cfg.batch)]))
     barrier(dist, device)
     clocks = sampler.stop()
+    if checks:
+        pending.append(pool.submit([(cfg, step, "delta", l, b) for step in checks for l in ld
+                                    for b in range(cfg.batch)]))
     lat = np.array([s.elapsed_time(e) * 1000.0 for s, e in events])
     us = max_over_ranks(dist, float(lat.mean()), device)
 

@@ -114,15 +114,15 @@ __device__ __noinline__ void select_final(const SelectFinal a, unsigned char* sm
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int j = jb + i * NTHR;
+            if (j >= N) break;   // small contexts: most slots are empty
+            acc[j] = 0ull;
             const float sc = __ull2float_rn(v[i]) * kFixInv;
+            if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
             const uint32_t key = order_key(sc);
-            const bool cand = (j >= sinkP) & (j < recStart);   // (implies j < N)
-            kmin = cand ? min(kmin, key) : kmin;
-            kmax = cand ? max(kmax, key) : kmax;
-            if (j < N) {
-                acc[j] = 0ull;
-                keys[j] = key;
-                if (a.page_scores != nullptr) a.page_scores[size_t(b) * maxp + j] = sc;
+            keys[j] = key;
+            if (j >= sinkP && j < recStart) {
+                kmin = min(kmin, key);
+                kmax = max(kmax, key);
             }
         }
     }
