@@ -73,8 +73,6 @@ struct MmaSmem {
     static constexpr size_t kBytes = 1024 /* alignment slack */ + kMain + kBars + kRecv;
 };
 
-constexpr int kPrefetchPages = 4;   // pages per warp beyond the stage ring prefetched into L2 up front
-
 template <int D, int G, int STAGES, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeParams p,
                                                               const __grid_constant__ CUtensorMap tmap_k,
@@ -166,21 +164,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
             if (ph >= 0 && (lp != ex.N - 1 || p.settled)) {
                 if (lane == 0) load_page(k, ph);
                 early |= 1u << k;
-            }
-        }
-        // The next pages beyond the stage ring into L2, so that their copies, issued as stages free
-        // up, do not wait a second full memory latency (L2 is the point of coherence: a page the
-        // previous kernel still writes is read correctly later).  Speculative lists are not used.
-        if (!speculative) {
-            const int npf = min(STAGES + kPrefetchPages, nk);
-            for (int k = STAGES; k < npf; ++k) {
-                int lp, ph;
-                pages_get(pages, k, lp, ph);
-                if (lane == 0 && ph >= 0) {
-                    const size_t off = (size_t(ph) * p.num_kv_heads + g) * (kPage * D);
-                    prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.k_pool) + off, kPage * D * 2);
-                    prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.v_pool) + off, kPage * D * 2);
-                }
             }
         }
     }
