@@ -49,8 +49,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     __syncwarp();
     merge_prologue(recv);
     // The page table and kv_len are inputs of the whole step (no kernel of the stream writes them),
-    // so full and delta layers resolve their pages before waiting for the previous kernel; the
-    // sparse layers' page list is the output of the delta-layer and is read after the wait.
+    // so full and delta layers resolve their pages before waiting for the previous kernel; a sparse
+    // layer's page list is the output of the delta-layer: read after the wait unless the caller
+    // states it settled.
     SeqExtent ex = seq_extent(p, b);
     int i0 = 0, nk = 0;
     WarpPages pages;
@@ -61,24 +62,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         nk = (i1 - i0 > warp) ? (i1 - i0 - warp + kWarps - 1) / kWarps : 0;   // pages of this warp
         pages_init(pages, p, ex, b, i0, warp, nk, lane);
     };
-    if (p.mode != kModeSparse) setup();
-    pdl_wait();      // q, the pools and the selection are written by earlier kernels
-    pdl_trigger();
-    if (p.mode == kModeSparse) setup();
-    const int n = ex.n;
-
-    // ---- queries of the group, pre-scaled into base-2 logits
-    float q[G][DS];
-    {
-        const T* qp = reinterpret_cast<const T*>(p.q) + (size_t(b) * Hq + h0) * D + hl * DS;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            load_row<T, DS>(qp + size_t(h) * D, q[h]);
-#pragma unroll
-            for (int d = 0; d < DS; ++d) q[h][d] *= p.qscale;
-        }
-    }
-
     const T* kpool = reinterpret_cast<const T*>(p.k_pool);
     const T* vpool = reinterpret_cast<const T*>(p.v_pool);
     const uint64_t policy = evict_first_policy();
@@ -99,7 +82,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             mbar_arrive(&wbar[s]);  // completes the phase with no data; consumers skip the page
         }
     };
-    for (int k = 0; k < min(STAGES, nk); ++k) issue(k);
+
+    // Before waiting for the previous kernel: full and delta layers (and sparse layers whose
+    // selection the caller states settled) know their pages, so the first stages' copies start
+    // now, except the page holding the appended token, which the previous kernel may still write
+    // (settled inputs: that one too); q goes to L2.
+    const bool known = p.mode != kModeSparse || p.settled;
+    uint32_t early = 0;   // bit k: page k's copy was issued before the wait
+    if (known) {
+        setup();
+        for (int k = 0; k < min(STAGES, nk); ++k) {
+            int lp, ph;
+            pages_get(pages, k, lp, ph);
+            if (ph >= 0 && (lp != ex.N - 1 || p.settled)) {
+                issue(k);
+                early |= 1u << k;
+            }
+        }
+    }
+    if (threadIdx.x == 0) prefetch_l2(reinterpret_cast<const T*>(p.q) + (size_t(b) * Hq + h0) * D, G * D * sizeof(T));
+    pdl_wait();      // q, the appended token and a selection written by earlier kernels
+    pdl_trigger();
+    if (!known) setup();
+    const int n = ex.n;
+
+    // ---- queries of the group, pre-scaled into base-2 logits
+    float q[G][DS];
+    {
+        const T* qp = reinterpret_cast<const T*>(p.q) + (size_t(b) * Hq + h0) * D + hl * DS;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            load_row<T, DS>(qp + size_t(h) * D, q[h]);
+#pragma unroll
+            for (int d = 0; d < DS; ++d) q[h][d] *= p.qscale;
+        }
+    }
+
+    for (int k = 0; k < min(STAGES, nk); ++k)
+        if (!((early >> k) & 1u)) issue(k);
 
     float m_run = -INFINITY, l_run = 0.f;  // running state of head (hl & (GP-1)) of this half
     float o[G][DS];
