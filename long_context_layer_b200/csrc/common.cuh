@@ -215,7 +215,6 @@ struct DecodeParams {
     unsigned long long* score_acc;   // [B][max_pages] page scores in 2^-44 fixed point, summed over the
                                      // KV heads by integer atomics; zero between launches
     uint32_t* keys;           // [B][max_pages] order keys of the page scores (when shared memory is short)
-    int* unit_tickets;        // [B][Hkv] CTAs of a unit that finished, zero between launches
     int* seq_tickets;         // [B] units of a sequence that finished, zero between launches
 };
 

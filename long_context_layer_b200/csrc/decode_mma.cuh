@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_mma_kernel(const DecodeP
     constexpr int kPart = STAGES * int(S::kPage) / 4;     // floats between two warps' records
     const float* mo0 = reinterpret_cast<const float*>(smem);
     float pre[2][G];   // delta-layers: this CTA's page terms, loaded before the merge
-    if (p.fuse_select && p.num_clusters == 1) select_preload<WARPS * 32, G>(p, b, g, ex.N, pre);
+    if (p.fuse_select) select_preload<WARPS * 32, G>(p, b, g, ex.N, pre);
     merge_epilogue<__nv_bfloat16, D, G, WARPS, WARPS * 32, kRow>(
         p, smem, mo0, mo0 + kMaxGroup * kRow, recv, b, g, kPart, kPart,
         (p.mode == kModeDelta) ? mo0 + kMaxGroup * kRow + kMaxGroup * 2 : nullptr);

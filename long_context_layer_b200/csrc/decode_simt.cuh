@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
     __syncthreads();
     float pre[2][G];   // delta-layers: this CTA's page terms, loaded before the merge
-    if (p.fuse_select && p.num_clusters == 1) select_preload<kThreads, G>(p, b, g, ex.N, pre);
+    if (p.fuse_select) select_preload<kThreads, G>(p, b, g, ex.N, pre);
     merge_epilogue<T, D, G, kWarps * 2>(p, smem, mo, mml, recv, b, g, kMaxGroup * D, kMaxGroup * 2);
     // delta-layers scoring with HEAD_SUM: page scores and the selection, in the stage area
     if (p.fuse_select) select_tail<kThreads, G, D>(p, smem, S::kMain, recv, b, g, ex.n, ex.N, pre);

@@ -55,7 +55,7 @@ enum : int { kVarNarrow = 0, kVarWide = 1, kVarShort = 2 };   // tensor-core ker
 constexpr int variant_threads(int v) { return 32 * (v == kVarWide ? kMmaWideWarps : v == kVarShort ? kMmaShortWarps : kWarps); }
 
 struct WsLayout {
-    size_t err, tickets, unit_tickets, seq_tickets, part_ml, part_o, page_lse, split_ml, score_acc, keys, logits,
+    size_t err, tickets, seq_tickets, part_ml, part_o, page_lse, split_ml, score_acc, keys, logits,
         total;
 };
 
@@ -212,7 +212,6 @@ WsLayout ws_layout(const delta_desc* d, int batch, int max_pages, bool with_logi
     // the counters (error word, tickets) come first: they are the part that must start at zero
     w.err = off;          off += align256(64);
     w.tickets = off;      off += align256(size_t(batch) * d->num_kv_heads * sizeof(int));
-    w.unit_tickets = off; off += align256(size_t(batch) * d->num_kv_heads * sizeof(int));
     w.seq_tickets = off;  off += align256(size_t(batch) * sizeof(int));
     w.part_ml = off;      off += align256(rows * S * sizeof(float2));
     w.part_o = off;       off += align256(rows * S * d->head_dim * sizeof(float));
@@ -573,6 +572,8 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     if (mode == kModeSparse && sel_stride_in < items) items = sel_stride_in;
     const SplitPlan plan = fit_plan(plan_splits(d->dtype, D, pt->batch, Hkv, items), d->dtype, D, Hq / Hkv,
                                     pt->batch * Hkv, items, mode == kModeDelta && !head_max);
+    // the in-kernel selection forms each unit's normalisers from its one cluster's merge
+    if (mode == kModeDelta && !head_max && plan.clusters != 1) return DELTA_ERR_UNSUPPORTED;
     const int S = plan.splits();
     unsigned char* base = static_cast<unsigned char*>(ws);
 
@@ -617,7 +618,6 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
         prm.page_scores = page_scores;
         prm.score_acc = reinterpret_cast<unsigned long long*>(base + L.score_acc);
         prm.keys = reinterpret_cast<uint32_t*>(base + L.keys);
-        prm.unit_tickets = reinterpret_cast<int*>(base + L.unit_tickets);
         prm.seq_tickets = reinterpret_cast<int*>(base + L.seq_tickets);
     }
 

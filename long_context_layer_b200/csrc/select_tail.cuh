@@ -8,15 +8,13 @@
 // = sum_h 2^(lse_hj - c_h), with lse_hj the log2-sum-exp of head h's base-2 logits on page j
 // (written by the decode loop) and c_h that head's log2-sum-exp over the whole context.
 //
-// No CTA waits for another.  When a (sequence, KV head) unit is one cluster, the output merge has
-// already given every CTA every split's state of the unit's heads, so each CTA forms c_h itself
-// and adds its own pages' share of the scores (the sum over the unit's G heads) into per-page
-// 2^-44 fixed-point accumulators with integer atomics (integer addition is associative, so the
-// sums do not depend on the order of arrival), then takes one ticket on its sequence.  When a
-// unit spans several clusters, each CTA takes a ticket on its unit first, and the unit's last CTA
-// forms c_h from the splits' states in the workspace and adds the unit's shares.  The last CTA of
-// the sequence reads the sums, finds the k-th largest candidate score by an adaptive-range radix
-// select and writes the ascending selection.
+// No CTA waits for another.  Delta-layer plans keep each (sequence, KV head) unit in one cluster,
+// so the output merge has already given every CTA every split's state of the unit's heads: each CTA
+// forms c_h itself and adds its own pages' share of the scores (the sum over the unit's G heads)
+// into per-page 2^-44 fixed-point accumulators with integer atomics (integer addition is
+// associative, so the sums do not depend on the order of arrival), then takes one ticket on its
+// sequence.  The last CTA of the sequence reads the sums, finds the k-th largest candidate score by
+// an adaptive-range radix select and writes the ascending selection.
 #pragma once
 
 #include "common.cuh"
@@ -344,8 +342,7 @@ template <int NTHR, int G, int D>
 __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char* smem, size_t free_bytes,
                                             const float* recv, int b, int g, int n, int N,
                                             const float (&pre)[2][G]) {
-    constexpr int W = NTHR / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, S = p.num_splits, h0 = g * G;
     const size_t maxp = size_t(p.max_pages);
     float* s_c = reinterpret_cast<float*>(smem);               // [kMaxGroup] per-head normalisers
@@ -378,54 +375,29 @@ __device__ __forceinline__ void select_tail(const DecodeParams& p, unsigned char
     // c_h = log2 of the sum over states of l * 2^m (no token of the head: +inf, every term 0)
     auto norm = [](float M, float Z) { return (Z > 0.f) ? M + log2_approx(Z) : INFINITY; };
 
-    if (p.num_clusters == 1) {
-        // every state of the unit is in this CTA's receive area: c_h here, then this CTA's pages
-        const int C = S;
-        const float* st = merge_recv_states<D, G>(recv, C);   // [C][G][4]: (m, l) then the fp32-term (m, l)
-        __syncthreads();   // no thread still reads the merge records in the stage area
-        if (tid < G) {
-            float M = -INFINITY;
-            for (int j = 0; j < C; ++j) M = fmaxf(M, st[(j * G + tid) * 4 + 2]);
-            const float mu = (M == -INFINITY) ? 0.f : M;
-            float Z = 0.f;
-            for (int j = 0; j < C; ++j) {
-                const float l = st[(j * G + tid) * 4 + 3];
-                if (l > 0.f) Z = fmaf(l, exp2_approx(st[(j * G + tid) * 4 + 2] - mu), Z);
-            }
-            s_c[tid] = norm(M, Z);
+    // Delta-layer plans keep each unit in one cluster (fit_plan), so every state of the unit is in
+    // this CTA's receive area: c_h here, then this CTA's pages
+    const int C = S;
+    const float* st = merge_recv_states<D, G>(recv, C);   // [C][G][4]: (m, l) then the fp32-term (m, l)
+    __syncthreads();   // no thread still reads the merge records in the stage area
+    if (tid < G) {
+        float M = -INFINITY;
+        for (int j = 0; j < C; ++j) M = fmaxf(M, st[(j * G + tid) * 4 + 2]);
+        const float mu = (M == -INFINITY) ? 0.f : M;
+        float Z = 0.f;
+        for (int j = 0; j < C; ++j) {
+            const float l = st[(j * G + tid) * 4 + 3];
+            if (l > 0.f) Z = fmaf(l, exp2_approx(st[(j * G + tid) * 4 + 2] - mu), Z);
         }
-        __syncthreads();
-        const int i0 = blockIdx.x * p.items_per_split, i1 = min(i0 + p.items_per_split, N);
-#pragma unroll
-        for (int i = 0; i < 2; ++i)   // the preloaded pages
-            if (i0 + tid + i * NTHR < i1) add_share(i0 + tid + i * NTHR, pre[i]);
-        shares(i0 + 2 * NTHR, i1);
-        if (!arrive_last(p.seq_tickets + b, Hkv * S, s_flag)) return;
-    } else {
-        // the unit's last CTA forms c_h from the splits' states and adds the unit's shares
-        if (!arrive_last(p.unit_tickets + b * Hkv + g, S, s_flag)) return;
-        for (int h = warp; h < G; h += W) {
-            const float2* ps = p.split_ml + (size_t(b) * Hq + h0 + h) * S;
-            float M = -INFINITY, Z = 0.f;
-            for (int base = 0; base < S; base += 32) {
-                const float2 v = (base + lane < S) ? __ldcg(ps + base + lane) : make_float2(-INFINITY, 0.f);
-                float Mr = v.x;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
-                const float Mn = fmaxf(M, Mr);
-                const float mu = (Mn == -INFINITY) ? 0.f : Mn;
-                float z = (v.y > 0.f) ? v.y * exp2_approx(v.x - mu) : 0.f;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-                Z = Z * exp2_approx(M - mu) + z;
-                M = Mn;
-            }
-            if (lane == 0) s_c[h] = norm(M, Z);
-        }
-        __syncthreads();
-        shares(0, N);
-        if (!arrive_last(p.seq_tickets + b, Hkv, s_flag)) return;
+        s_c[tid] = norm(M, Z);
     }
+    __syncthreads();
+    const int i0 = blockIdx.x * p.items_per_split, i1 = min(i0 + p.items_per_split, N);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)   // the preloaded pages
+        if (i0 + tid + i * NTHR < i1) add_share(i0 + tid + i * NTHR, pre[i]);
+    shares(i0 + 2 * NTHR, i1);
+    if (!arrive_last(p.seq_tickets + b, Hkv * S, s_flag)) return;
     SelectFinal a;
     a.score_acc = p.score_acc;
     a.keys = p.keys;
