@@ -92,14 +92,14 @@ class DeltaStack:
                   out_dev, append: bool = True, early_layers: int = 2, out_chunks: int = 8):
         """One decode step whose inputs and outputs live in (pinned) host memory.
 
-        On a copy stream: the first `early_layers` layers' q and the appended tokens (every
-        layer's append needs them), then the other layers' q, which arrive while the first
-        layers compute.  The outputs return to the host on another stream in `out_chunks`
-        groups of consecutive layers, each as soon as its last layer is done.  The compute
-        stream joins the copy streams at those few points only, so most consecutive kernels keep
-        their programmatic-launch overlap.  *_dev are device staging buffers of the same shapes.
-        Everything is enqueued on the current stream (graph-capturable); out_host is complete
-        once that stream reaches the end of the step.
+        On a copy stream: the first `early_layers` layers' q and appended tokens, then every other
+        layer's, which arrive while the first layers compute (the append runs as two launches, one
+        per group of layers).  The outputs return to the host on another stream in `out_chunks`
+        groups of consecutive layers, each as soon as its last layer is done.  The compute stream
+        joins the copy streams at those few points only, so most consecutive kernels keep their
+        programmatic-launch overlap.  *_dev are device staging buffers of the same shapes.
+        Everything is enqueued on the current stream (graph-capturable); out_host is complete once
+        that stream reaches the end of the step.
         """
         main = torch.cuda.current_stream(self.device)
         if not hasattr(self, "_up"):
@@ -110,36 +110,35 @@ class DeltaStack:
         early = max(1, min(early_layers, L))
         up.wait_stream(main)
         down.wait_stream(main)
+        groups = [(0, early)] + ([(early, L)] if early < L else [])
+        ready = []
         with torch.cuda.stream(up):
-            q_dev[:early].copy_(q_host[:early], non_blocking=True)
-            k_new_dev.copy_(k_new_host, non_blocking=True)
-            v_new_dev.copy_(v_new_host, non_blocking=True)
-            first_ready = torch.cuda.Event()
-            first_ready.record(up)
-            rest_ready = None
-            if early < L:
-                q_dev[early:].copy_(q_host[early:], non_blocking=True)
-                rest_ready = torch.cuda.Event()
-                rest_ready.record(up)
-        main.wait_event(first_ready)
+            for a, b in groups:
+                q_dev[a:b].copy_(q_host[a:b], non_blocking=True)
+                k_new_dev[a:b].copy_(k_new_host[a:b], non_blocking=True)
+                v_new_dev[a:b].copy_(v_new_host[a:b], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(up)
+                ready.append(ev)
         st = main.cuda_stream
-        if append:
-            N.kv_append_layers(self.desc, self.pt, k_new_dev, v_new_dev, k_pools, v_pools, st)
         per = -(-L // max(1, out_chunks))
         cur, c0 = -1, 0
-        for l, kind in enumerate(self.kinds):
-            if l == early and rest_ready is not None:
-                main.wait_event(rest_ready)
-            self._layer(l, kind, cur, q_dev, k_pools, v_pools, out_dev, st)
-            if kind == DELTA:
-                cur = self.delta_layers.index(l)
-            if l + 1 - c0 == per or l == L - 1:
-                done = torch.cuda.Event()
-                done.record(main)
-                down.wait_event(done)
-                with torch.cuda.stream(down):
-                    out_host[c0:l + 1].copy_(out_dev[c0:l + 1], non_blocking=True)
-                c0 = l + 1
+        for gi, (a, b) in enumerate(groups):
+            main.wait_event(ready[gi])
+            if append:
+                N.kv_append_layers(self.desc, self.pt, k_new_dev[a:b], v_new_dev[a:b], k_pools[a:b], v_pools[a:b], st)
+            for l in range(a, b):
+                kind = self.kinds[l]
+                self._layer(l, kind, cur, q_dev, k_pools, v_pools, out_dev, st)
+                if kind == DELTA:
+                    cur = self.delta_layers.index(l)
+                if l + 1 - c0 == per or l == L - 1:
+                    done = torch.cuda.Event()
+                    done.record(main)
+                    down.wait_event(done)
+                    with torch.cuda.stream(down):
+                        out_host[c0:l + 1].copy_(out_dev[c0:l + 1], non_blocking=True)
+                    c0 = l + 1
         main.wait_stream(up)
         main.wait_stream(down)
 
