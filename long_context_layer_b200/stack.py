@@ -94,8 +94,9 @@ class DeltaStack:
 
         On a copy stream: the first `early_layers` layers' q and appended tokens, then every other
         layer's, which arrive while the first layers compute (the append runs as two launches, one
-        per group of layers).  The outputs return to the host on another stream in `out_chunks`
-        groups of consecutive layers, each as soon as its last layer is done.  The compute stream
+        per group of layers).  The outputs return to the host on another stream in about `out_chunks`
+        groups of consecutive layers, each as soon as its last layer is done (the last layer on its
+        own, so that only its output is copied after the final kernel).  The compute stream
         joins the copy streams at those few points only, so most consecutive kernels keep their
         programmatic-launch overlap.  *_dev are device staging buffers of the same shapes.
         Everything is enqueued on the current stream (graph-capturable); out_host is complete once
@@ -121,7 +122,7 @@ class DeltaStack:
                 ev.record(up)
                 ready.append(ev)
         st = main.cuda_stream
-        per = -(-L // max(1, out_chunks))
+        per = -(-max(L - 1, 1) // max(1, out_chunks))
         cur, c0 = -1, 0
         for gi, (a, b) in enumerate(groups):
             main.wait_event(ready[gi])
@@ -132,7 +133,7 @@ class DeltaStack:
                 self._layer(l, kind, cur, q_dev, k_pools, v_pools, out_dev, st)
                 if kind == DELTA:
                     cur = self.delta_layers.index(l)
-                if l + 1 - c0 == per or l == L - 1:
+                if l + 1 - c0 == per or l >= L - 2:
                     done = torch.cuda.Event()
                     done.record(main)
                     down.wait_event(done)
