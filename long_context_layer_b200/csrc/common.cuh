@@ -212,7 +212,7 @@ struct DecodeParams {
     int32_t* sel_pages_out;   // [B][sel_stride_out]
     int32_t sel_stride_out;
     float* page_scores;       // [B][max_pages] or null
-    unsigned long long* score_acc;   // [B][max_pages] page scores in 2^-44 fixed point, summed over the
+    unsigned long long* score_acc;   // [B][max_pages] page scores in 2^-55 fixed point, summed over the
                                      // KV heads by integer atomics; zero between launches
     uint32_t* keys;           // [B][max_pages] order keys of the page scores (when shared memory is short)
     int* seq_tickets;         // [B] units of a sequence that finished, zero between launches

@@ -11,7 +11,7 @@
 // No CTA waits for another.  Delta-layer plans keep each (sequence, KV head) unit in one cluster,
 // so the output merge has already given every CTA every split's state of the unit's heads: each CTA
 // forms c_h itself and adds its own pages' share of the scores (the sum over the unit's G heads)
-// into per-page 2^-44 fixed-point accumulators with integer atomics (integer addition is
+// into per-page 2^-55 fixed-point accumulators with integer atomics (integer addition is
 // associative, so the sums do not depend on the order of arrival), then takes one ticket on its
 // sequence.  The last CTA of the sequence reads the sums, finds the k-th largest candidate score by
 // an adaptive-range radix select and writes the ascending selection.
@@ -22,8 +22,11 @@
 namespace delta {
 
 constexpr int kTailList = 128;              // keys the final rank step compares pairwise, at most
-constexpr float kFixScale = 17592186044416.f;   // 2^44: fixed-point unit of the score accumulators
-constexpr float kFixInv = 5.684341886080802e-14f;   // 2^-44
+// Fixed-point unit of the score accumulators: 2^-55.  A page score is at most H_q <= 256 = 2^8
+// (delta-layers are limited to 256 query heads), so every sum stays below 2^63; scores resolve down
+// to 2^-55 (about 2.8e-17), below which a page scores 0 and ties go to the lower page index.
+constexpr float kFixScale = 36028797018963968.f;   // 2^55
+constexpr float kFixInv = 2.7755575615628914e-17f;  // 2^-55
 
 // What the sequence's last CTA needs (passed by value to the non-inlined final stage).
 struct SelectFinal {

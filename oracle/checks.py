@@ -1,9 +1,14 @@
 """Comparison of a GPU page selection with the oracle's — TEST INFRASTRUCTURE ONLY.
 
 Selections are compared exactly, except where the oracle's k-th and (k+1)-th candidate
-scores lie within ``TIE_REL`` (relative) of each other: pages inside that near-tied band may
-be swapped, since rounding in a different summation order may legitimately reorder them.
-Every page outside the band, the sink pages and the recency pages must agree exactly.
+scores lie within ``TIE_REL`` (relative) plus ``TIE_ABS`` (absolute) of each other: pages
+inside that near-tied band may be swapped, since rounding in a different summation order may
+legitimately reorder them.  Every page outside the band, the sink pages and the recency pages
+must agree exactly.
+
+``TIE_ABS`` is the GPU selection's resolution: it sums each page's score in fixed point with
+unit 2^-55, every KV head's share rounded on its own (at most 32 KV heads, so at most 2^-51
+of rounding per page), which cannot order two scores closer than that; 2^-50 covers it.
 """
 from __future__ import annotations
 
@@ -12,6 +17,7 @@ import numpy as np
 from . import delta_oracle as O
 
 TIE_REL = 1e-4
+TIE_ABS = 2.0 ** -50
 
 
 def selection_ok(gpu_sel, S_oracle: np.ndarray, n: int, budget_pages: int, sink_tokens: int,
@@ -33,9 +39,10 @@ def selection_ok(gpu_sel, S_oracle: np.ndarray, n: int, budget_pages: int, sink_
         return False, False, ref
     kth = S_oracle[cands[budget_pages - 1]]
     nxt = S_oracle[cands[budget_pages]]
-    if abs(kth - nxt) >= TIE_REL * abs(kth):
+    band = TIE_REL * abs(kth) + TIE_ABS
+    if abs(kth - nxt) >= band:
         return False, False, ref
-    tied = {j for j in cands if abs(S_oracle[j] - kth) < TIE_REL * abs(kth)}
+    tied = {j for j in cands if abs(S_oracle[j] - kth) < band}
     if not forced <= set(gpu_sel):
         return False, False, ref
     sure = set(ref) - tied

@@ -4,7 +4,7 @@ from __future__ import annotations
 import numpy as np
 
 from oracle import delta_oracle as O  # noqa: F401
-from oracle.checks import TIE_REL, selection_ok  # noqa: F401  (one definition for tests and bench)
+from oracle.checks import TIE_ABS, TIE_REL, selection_ok  # noqa: F401  (one definition for tests and bench)
 from synth import rng
 
 # Output tolerances (stated with the workloads): fp32 max-abs <= 1e-5;
