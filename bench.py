@@ -749,7 +749,8 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
         check = {"selection_match_rate": round(ok / total, 4), "selections_checked": total,
                  "selections_exact": exact, "steps_checked": checks,
                  "rule": "every delta-layer x every sequence at each checked step; a match is the oracle's set, "
-                         "pages swapped only inside a band of scores within 1e-4 relative of the k-th",
+                         "pages swapped only inside a band of scores within 1e-4 relative plus 2^-50 absolute "
+                         "of the k-th",
                  "delta_output_max_abs_err": round(worst_abs, 6), "delta_output_max_rel_l2": round(worst_rel, 6)}
     elif pool is not None:
         pool.close()

@@ -9,7 +9,8 @@ from synth import rng
 
 # Output tolerances (stated with the workloads): fp32 max-abs <= 1e-5;
 # bf16 max-abs <= 2e-2 and relative L2 <= 5e-3.  Near-tie rule for selections: sets must be
-# identical unless the oracle's k-th and (k+1)-th candidate scores differ by < 1e-4 relative.
+# identical unless the oracle's k-th and (k+1)-th candidate scores differ by < 1e-4 relative
+# plus 2^-50 absolute (the GPU's fixed-point score resolution).
 F32_MAX_ABS = 1e-5
 BF16_MAX_ABS = 2e-2
 BF16_REL_L2 = 5e-3
