@@ -651,6 +651,52 @@ def check_points(cfg, m: int) -> list:
     return pts if m < 0 else pts[:m]
 
 
+def selection_quality(cfg, case, layers, cnt, pages) -> dict:
+    """How the GPU's selections behave along the trajectory: the fraction of each step's selected
+    pages that the previous step also selected (per delta-layer and sequence), and the fraction of
+    the planted keys' pages that the selection in force covers, for every layer it serves (the
+    delta-layer itself and the sparse layers after it).  cnt [T, n_delta, B], pages [T, n_delta, B, stride]."""
+    import numpy as np
+    T, nd, B, stride = pages.shape
+    P, de = cfg.page_size, cfg.drift_every or T
+    mask = np.zeros((T, nd, B, case.max_pages_per_seq), dtype=bool)
+    t, i, b, s = np.nonzero(np.arange(stride)[None, None, None, :] < cnt[..., None])
+    mask[t, i, b, np.clip(pages[t, i, b, s], 0, case.max_pages_per_seq - 1)] = True
+    res = {}
+    if T > 1:
+        ov = (mask[1:] & mask[:-1]).sum(-1) / np.maximum(mask[1:].sum(-1), 1)   # [T-1, nd, B]
+        moved = np.array([(k + 1) % de == 0 for k in range(T - 1)])
+        res["step_overlap"] = {"mean": round(float(ov.mean()), 4), "min": round(float(ov.min()), 4),
+                               "mean_at_drift_steps": round(float(ov[moved].mean()), 4) if moved.any() else None,
+                               "mean_other_steps": round(float(ov[~moved].mean()), 4)}
+    served = [range(l, layers[k + 1] if k + 1 < nd else cfg.num_layers) for k, l in enumerate(layers)]
+    rec_all, rec_delta, rec_first = [], [], []
+    for t0 in range(0, T, de):
+        t1 = min(t0 + de, T)
+        for k in range(nd):
+            for l in served[k]:
+                for bb in range(B):
+                    pos = [case.planted_positions(l, bb, g, t0) for g in range(cfg.num_kv_heads)]
+                    pp = np.unique(np.concatenate(pos) // P) if pos else np.zeros(0, dtype=np.int64)
+                    if len(pp) == 0:
+                        continue
+                    r = mask[t0:t1, k, bb][:, pp].mean(axis=1)   # per step
+                    rec_all.append(r)
+                    if l == layers[k]:
+                        rec_delta.append(r)
+                    rec_first.append(r[:1])
+    if rec_all:
+        res["planted_page_recall"] = {
+            "served_layers_mean": round(float(np.concatenate(rec_all).mean()), 4),
+            "served_layers_min": round(float(np.concatenate(rec_all).min()), 4),
+            "delta_layers_mean": round(float(np.concatenate(rec_delta).mean()), 4),
+            "first_step_after_each_drift_mean": round(float(np.concatenate(rec_first).mean()), 4)}
+    res["how"] = ("every step's selections copied to pinned host memory after the step (outside the timed "
+                  "region); overlap = |sel_t & sel_t-1| / |sel_t|; recall = share of the pages holding a "
+                  "layer's planted keys (all KV heads) inside the selection that layer uses")
+    return res
+
+
 def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
     """The drifting trajectory: every decode step replays one CUDA graph; between steps (untimed)
     the cache grows by one token per sequence and, every drift_every steps, the planted keys move."""
@@ -700,6 +746,8 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
     timed = set(timed_steps)
     events, pending, gpu_sel, gpu_out = [], [], {}, {}
     ld = stack.delta_layers
+    hist_cnt = torch.empty((T, len(ld), cfg.batch), dtype=torch.int32, pin_memory=True)
+    hist_pages = torch.empty((T, len(ld), cfg.batch, stack.sel_stride), dtype=torch.int32, pin_memory=True)
     for step in range(T):
         tr.prepare(step)
         if step in timed:
@@ -711,6 +759,8 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
             events.append((s0, s1))
         else:
             g.replay()
+        hist_cnt[step].copy_(stack.sel_cnt, non_blocking=True)    # after the step's end event
+        hist_pages[step].copy_(stack.sel_pages, non_blocking=True)
         if step in checks:   # copies only: the oracle runs after the timed loop (host cores stay free)
             cnt = stack.sel_cnt.cpu().numpy()
             pages = stack.sel_pages.cpu().numpy()
@@ -755,6 +805,7 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
     elif pool is not None:
         pool.close()
 
+    quality = selection_quality(cfg, case0, ld, hist_cnt.numpy(), hist_pages.numpy()) if ld else None
     tok = [attended_tokens(cfg, tr.case_at(s)) for s in (0, T - 1)]
     n_sparse = cfg.layer_kinds().count("sparse")
     km["roofline"]["share_of_step"] = round(n_sparse * km["roofline"]["us_per_launch"] / us_delta0, 3)
@@ -763,7 +814,8 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
         "trajectory": {"per_step_us": {"mean": round(float(lat.mean()), 3), "median": round(float(np.median(lat)), 3),
                                        "p99": round(float(np.percentile(lat, 99)), 3),
                                        "first": round(float(lat[0]), 3), "last": round(float(lat[-1]), 3)},
-                       "timed_steps": len(timed_steps), "steps_run": T, "oracle_check": check},
+                       "timed_steps": len(timed_steps), "steps_run": T, "oracle_check": check,
+                       "selection_quality": quality},
         "step0_us": round(us_delta0, 3), "full_stack_us": round(us_full0, 3),
         "speedup_vs_full_stack": round(us_full0 / us_delta0, 3),
         "attended_token_reduction": round(statistics.mean(t[1] / t[0] for t in tok), 3),

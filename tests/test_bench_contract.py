@@ -76,3 +76,39 @@ def test_trajectory_check_points_straddle_every_drift_boundary():
         assert s - 1 in pts and s in pts
     assert bench.check_points(C.DRIFT_48L, 3) == [0, 99, 100]
     assert bench.check_points(C.DRIFT_48L, 0) == []
+
+
+def test_selection_quality_overlap_and_planted_recall():
+    import dataclasses
+    import bench
+    cfg = dataclasses.replace(C.DRIFT_48L, batch=2, num_layers=8, steps=6, drift_every=3)
+    case = Case(cfg, step=0)
+    layers = [2, 5]
+    T, nd, B, N = cfg.steps, len(layers), cfg.batch, case.max_pages_per_seq
+    stride = N
+    # every page selected at every step: overlap 1, recall 1
+    cnt = np.full((T, nd, B), N, dtype=np.int32)
+    pages = np.broadcast_to(np.arange(N, dtype=np.int32), (T, nd, B, N)).copy()
+    q = bench.selection_quality(cfg, case, layers, cnt, pages)
+    assert q["step_overlap"]["mean"] == 1.0 and q["planted_page_recall"]["served_layers_mean"] == 1.0
+    # only the sink page: planted keys lie past the sink tokens, so recall is 0
+    cnt1 = np.ones((T, nd, B), dtype=np.int32)
+    pages1 = np.zeros((T, nd, B, stride), dtype=np.int32)
+    q = bench.selection_quality(cfg, case, layers, cnt1, pages1)
+    assert q["planted_page_recall"]["served_layers_mean"] == 0.0 and q["step_overlap"]["min"] == 1.0
+    # exactly the delta-layer's own planted pages at each step: its recall is 1; the selection
+    # changes at the drift step (3), where the overlap drops
+    cnt2 = np.zeros((T, nd, B), dtype=np.int32)
+    pages2 = np.zeros((T, nd, B, stride), dtype=np.int32)
+    for t in range(T):
+        for k, l in enumerate(layers):
+            for b in range(B):
+                pos = np.concatenate([case.planted_positions(l, b, g, t) for g in range(cfg.num_kv_heads)])
+                pp = np.unique(pos // cfg.page_size)
+                cnt2[t, k, b] = len(pp)
+                pages2[t, k, b, :len(pp)] = pp
+    q = bench.selection_quality(cfg, case, layers, cnt2, pages2)
+    r = q["planted_page_recall"]
+    assert r["delta_layers_mean"] == 1.0 and 0.0 < r["served_layers_mean"] < 1.0
+    ov = q["step_overlap"]
+    assert ov["mean_other_steps"] == 1.0 and ov["mean_at_drift_steps"] < 1.0
