@@ -53,6 +53,9 @@ def parse(argv=None):
                     help="trajectory steps whose delta-layer selections (every sequence) the oracle checks: "
                          "-1 every step at a drift boundary (0, 99, 100, ..., last), 0 none, m the first m of those")
     ap.add_argument("--oracle-procs", type=int, default=0, help="oracle worker processes (0: every host core)")
+    ap.add_argument("--check-every-step", action="store_true",
+                    help="trajectory: also check every step's delta-layer selections against the oracle "
+                         "(minutes of host CPU after the timed loop)")
     ap.add_argument("--no-extra", action="store_true", help="skip the summaries of the 64k and 8k workloads")
     ap.add_argument("--print-source-hash", action="store_true", help="print the kernel-source hash and exit")
     ap.add_argument("--reduce", choices=["sum", "max"], default="sum",
@@ -708,8 +711,9 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
     K = min(args.steps, T) if args.steps else T
     timed_steps = sorted({int(round(i * (T - 1) / max(K - 1, 1))) for i in range(K)}) if K > 1 else [0]
     checks = check_points(cfg, args.checks) if rank == 0 else []
+    every_step = rank == 0 and args.check_every_step and bool(cfg.delta_layers)
     pool = None
-    if checks:
+    if checks or every_step:
         from oracle.parallel import OraclePool
         pool = OraclePool(args.oracle_procs or None)   # spawn-started: safe after CUDA init
 
@@ -795,14 +799,38 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
                 o = gpu_out[(step, l, b)].astype(np.float64)
                 worst_abs = max(worst_abs, float(np.abs(o - o_ref).max()))
                 worst_rel = max(worst_rel, float(np.linalg.norm(o - o_ref) / max(np.linalg.norm(o_ref), 1e-30)))
-        pool.close()
         check = {"selection_match_rate": round(ok / total, 4), "selections_checked": total,
                  "selections_exact": exact, "steps_checked": checks,
                  "rule": "every delta-layer x every sequence at each checked step; a match is the oracle's set, "
                          "pages swapped only inside a band of scores within 1e-4 relative plus 2^-50 absolute "
                          "of the k-th",
                  "delta_output_max_abs_err": round(worst_abs, 6), "delta_output_max_rel_l2": round(worst_rel, 6)}
-    elif pool is not None:
+    every = None
+    if every_step:
+        from oracle.checks import selection_ok
+        t_chk = time.time()
+        de = cfg.drift_every or T
+        jobs = [(cfg, min(t0 + de, T) - 1, "delta_block", l, b, list(range(t0, min(t0 + de, T))))
+                for t0 in range(0, T, de) for l in ld for b in range(cfg.batch)]
+        ok = exact = total = 0
+        bad = []
+        for job, scores in pool.imap(jobs):
+            _, _, _, l, b, steps = job
+            i = ld.index(l)
+            for t, S in zip(steps, scores):
+                n = int(cfg.contexts(t)[b])
+                sel = hist_pages[t, i, b, :int(hist_cnt[t, i, b])].tolist()
+                good, ex, _ = selection_ok(sel, S, n, cfg.budget_pages, cfg.sink_tokens, cfg.recency_tokens,
+                                           cfg.page_size)
+                ok += int(good)
+                exact += int(ex)
+                total += 1
+                if not good and len(bad) < 8:
+                    bad.append({"step": t, "layer": l, "b": b})
+        every = {"selection_match_rate": round(ok / max(total, 1), 4), "selections_checked": total,
+                 "selections_exact": exact, "steps": T, "mismatches": bad,
+                 "host_seconds": round(time.time() - t_chk, 1)}
+    if pool is not None:
         pool.close()
 
     quality = selection_quality(cfg, case0, ld, hist_cnt.numpy(), hist_pages.numpy()) if ld else None
@@ -815,7 +843,7 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
                                        "p99": round(float(np.percentile(lat, 99)), 3),
                                        "first": round(float(lat[0]), 3), "last": round(float(lat[-1]), 3)},
                        "timed_steps": len(timed_steps), "steps_run": T, "oracle_check": check,
-                       "selection_quality": quality},
+                       "selection_quality": quality, "every_step_check": every},
         "step0_us": round(us_delta0, 3), "full_stack_us": round(us_full0, 3),
         "speedup_vs_full_stack": round(us_full0 / us_delta0, 3),
         "attended_token_reduction": round(statistics.mean(t[1] / t[0] for t in tok), 3),

@@ -6,7 +6,11 @@ step, with the planted keys of that step, and evaluates the plain fp64 oracle on
 
 * ``("full", layer, b)``           -> o [Hq, D] of dense attention;
 * ``("delta", layer, b)``          -> (o [Hq, D], S [pages]) dense attention and page scores;
-* ``("sparse", layer, b, pages)``  -> o [Hq, D] of attention over the given pages.
+* ``("sparse", layer, b, pages)``  -> o [Hq, D] of attention over the given pages;
+* ``("delta_block", layer, b, steps)`` -> [S at each of ``steps``]: page scores at several steps of
+  one drift block (the job's own step is the block's last).  Inside a block the planted keys stay
+  put and each step only appends a token, so the K and V of an earlier step are a prefix of the last
+  step's: they are regenerated once and every step's scores use its own context length.
 
 The pool uses the ``spawn`` start method, so it may be created after CUDA was initialised in the
 parent.  Nothing here reads GPU results: jobs carry only workload coordinates.
@@ -54,6 +58,16 @@ def run_job(job):
         return job, (o, O.page_scores(p, cfg.page_size))
     if kind == "sparse":
         return job, O.sparse_attention(q, K, V, list(job[5]), cfg.page_size)
+    if kind == "delta_block":
+        de = cfg.drift_every or (step + 1)
+        out = []
+        for t in job[5]:
+            if not (t <= step and t // de == step // de):
+                raise ValueError("delta_block: steps must lie in the block of the job's step, at or before it")
+            n = int(cfg.contexts(t)[b])
+            _, p = O.full_attention(q, K[:, :n], V[:, :n])
+            out.append(O.page_scores(p, cfg.page_size))
+        return job, out
     raise ValueError(kind)
 
 
@@ -76,6 +90,10 @@ class OraclePool:
 
     def submit(self, jobs):
         return self.pool.map_async(run_job, list(jobs), chunksize=1)
+
+    def imap(self, jobs):
+        """Results as they finish, in any order (each a (job, result) pair)."""
+        return self.pool.imap_unordered(run_job, list(jobs), chunksize=1)
 
     def run(self, jobs):
         return self.submit(jobs).get()
