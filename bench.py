@@ -635,6 +635,7 @@ def run_static(args, cfg, dist, rank, world, device, headline: bool = True) -> d
         res["gpu_launches"] = delta_stack.launches_per_step() * K
         res["cpu_baseline"] = (cpu_baseline_leg(cfg, case, args.cpu_seconds)
                                if rank == 0 and world == 1 and not args.no_cpu_baseline else None)
+        res["planted_logit_boost"] = planted_logit_boost(cfg, case, sorted(cfg.delta_layers))
     del g_delta, g_full
     delta_stack.graph = None
     full_stack.graph = None
@@ -652,6 +653,34 @@ def check_points(cfg, m: int) -> list:
             pts.update((s - 1, s))
     pts = sorted(pts)
     return pts if m < 0 else pts[:m]
+
+
+def planted_logit_boost(cfg, case, layers, sample: int = 256) -> dict | None:
+    """The synthetic workload's planted-key strength, measured on its stored values: the mean rise of
+    the scaled logit q_h . k / sqrt(D) that planting gives a key (planted row against the same
+    position's unplanted generator row, over the G query heads of its KV head), and the standard
+    deviation of the unplanted logits (the first `sample` positions), for the given layers."""
+    import numpy as np
+    from synth import rng
+    if cfg.planted == 0 or not layers:
+        return None
+    G, D = cfg.group, cfg.head_dim
+    sc = 1.0 / np.sqrt(D)
+    rises, spread = [], []
+    for l in layers:
+        q = case.q(l).astype(np.float64)
+        for b in range(cfg.batch):
+            for g in range(cfg.num_kv_heads):
+                qg = q[b, g * G:(g + 1) * G]
+                pos, rows = case.planted_rows(l, b, g)
+                if pos.size:
+                    base = case.kv_base(rng.T_K, l, b, g, pos).astype(np.float64)
+                    rises.append(((rows.astype(np.float64) - base) @ qg.T * sc).ravel())
+                ref = case.kv_base(rng.T_K, l, b, g, np.arange(min(sample, int(case.n[b])))).astype(np.float64)
+                spread.append((ref @ qg.T * sc).std(axis=0))
+    return {"mean_rise_nats": round(float(np.concatenate(rises).mean()), 3) if rises else None,
+            "unplanted_logit_std": round(float(np.concatenate(spread).mean()), 3),
+            "layers": list(layers)}
 
 
 def selection_quality(cfg, case, layers, cnt, pages) -> dict:
@@ -843,7 +872,8 @@ def run_trajectory(args, cfg, dist, rank, world, device) -> dict:
                                        "p99": round(float(np.percentile(lat, 99)), 3),
                                        "first": round(float(lat[0]), 3), "last": round(float(lat[-1]), 3)},
                        "timed_steps": len(timed_steps), "steps_run": T, "oracle_check": check,
-                       "selection_quality": quality, "every_step_check": every},
+                       "selection_quality": quality, "every_step_check": every,
+                       "planted_logit_boost": planted_logit_boost(cfg, case0, ld)},
         "step0_us": round(us_delta0, 3), "full_stack_us": round(us_full0, 3),
         "speedup_vs_full_stack": round(us_full0 / us_delta0, 3),
         "attended_token_reduction": round(statistics.mean(t[1] / t[0] for t in tok), 3),
