@@ -176,7 +176,8 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, int vari
     return pl;
 }
 
-SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
+// delta_fused: a delta-layer that scores and selects its pages inside the decode (HEAD_SUM).
+SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items, bool delta_fused = false) {
     // Few (sequence, KV head) units, so that a full cluster per unit fits one CTA per SM, and at
     // least two pages per warp of such a cluster: 8-warp CTAs, each warp streaming half the pages
     // of a 4-warp CTA's warp (the per-warp chain of dependent MMAs, exponentials and shuffles,
@@ -186,19 +187,25 @@ SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items) {
                       items >= 16 * kMmaWideWarps * 2;
     if (wide) return plan_variant(dtype, D, batch, Hkv, items, kVarWide);
     // 6 warps with 2 stages each (the same shared memory and pages in flight as 4 warps x 3 stages,
-    // spread over more warps) for two kinds of list:
+    // spread over more warps) for three kinds of list:
     //  - lists that 4-warp CTAs would cover with at most two pages per warp (a sparse layer of a
     //    small batch), so more warps share the few pages;
     //  - short lists (sparse layers, at most kShortListPages) that still give a 4-warp CTA at least
     //    kShortLongCta pages (a sparse layer of a large batch): each warp streams fewer pages, so the
     //    slowest warp, which ends the layer, finishes sooner (measured: 29.0 instead of 30.1 us per
     //    sparse layer of the 16-sequence 16k stack with 81 pages per CTA; slower at 32 pages per CTA
-    //    on the 4-sequence 64k stack, 17.2 instead of 16.0 us).  Long lists (full and delta layers)
-    //    keep 3 stages per warp.
+    //    on the 4-sequence 64k stack, 17.2 instead of 16.0 us);
+    //  - delta-layers of large batches (at most two splits per unit, at least 64 pages per CTA): the
+    //    page terms add work to every page, which more warps share (measured: 167 instead of 171 us
+    //    per delta-layer of the 16-sequence 16k stack; at nine splits per unit, the 64k stack's, the
+    //    6-warp plan ran slower, 204 instead of 178 us).
+    //  Other long lists (full layers) keep 3 stages per warp.
     constexpr int kShortListPages = 512, kShortLongCta = 48;
     const SplitPlan narrow = plan_variant(dtype, D, batch, Hkv, items, kVarNarrow);
     const int per_cta = (items + narrow.splits() - 1) / narrow.splits();
-    if (dtype == DELTA_BF16 && (per_cta <= 2 * kWarps || (items <= kShortListPages && per_cta >= kShortLongCta)))
+    const bool short_list = per_cta <= 2 * kWarps || (items <= kShortListPages && per_cta >= kShortLongCta);
+    const bool delta_large_batch = delta_fused && narrow.splits() <= 2 && per_cta >= 64;
+    if (dtype == DELTA_BF16 && (short_list || delta_large_batch))
         return plan_variant(dtype, D, batch, Hkv, items, kVarShort);
     return narrow;
 }
@@ -580,7 +587,7 @@ delta_status run_attention(int mode, const delta_desc* d, const delta_page_table
     const int D = d->head_dim, Hq = d->num_q_heads, Hkv = d->num_kv_heads;
     int items = pt->max_pages_per_seq;
     if (mode == kModeSparse && sel_stride_in < items) items = sel_stride_in;
-    const SplitPlan plan = fit_plan(plan_splits(d->dtype, D, pt->batch, Hkv, items), d->dtype, D, Hq / Hkv,
+    const SplitPlan plan = fit_plan(plan_splits(d->dtype, D, pt->batch, Hkv, items, mode == kModeDelta && !head_max), d->dtype, D, Hq / Hkv,
                                     pt->batch * Hkv, items, mode == kModeDelta && !head_max);
     // the in-kernel selection forms each unit's normalisers from its one cluster's merge
     if (mode == kModeDelta && !head_max && plan.clusters != 1) return DELTA_ERR_UNSUPPORTED;
