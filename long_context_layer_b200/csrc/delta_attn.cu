@@ -178,13 +178,20 @@ SplitPlan plan_variant(int dtype, int D, int batch, int Hkv, int items, int vari
 
 // delta_fused: a delta-layer that scores and selects its pages inside the decode (HEAD_SUM).
 SplitPlan plan_splits(int dtype, int D, int batch, int Hkv, int items, bool delta_fused = false) {
-    // Few (sequence, KV head) units, so that a full cluster per unit fits one CTA per SM, and at
-    // least two pages per warp of such a cluster: 8-warp CTAs, each warp streaming half the pages
-    // of a 4-warp CTA's warp (the per-warp chain of dependent MMAs, exponentials and shuffles,
-    // not the memory system, bounds such layers).  Short page lists (sparse layers) keep 4-warp
-    // CTAs, two per SM, so the next layer's CTAs find room beside them and start their loads.
-    const bool wide = DELTA_WIDE && dtype == DELTA_BF16 && int64_t(batch) * Hkv * 16 <= device_sm_count() &&
-                      items >= 16 * kMmaWideWarps * 2;
+    // One 8-warp CTA per SM, each warp streaming half the pages of a 4-warp CTA's warp (the per-warp
+    // chain of dependent MMAs, exponentials and shuffles, not the memory system, bounds such layers):
+    //  - few (sequence, KV head) units, so that a full cluster per unit fits one CTA per SM, and at
+    //    least two pages per warp of such a cluster (short lists of such batches, sparse layers, keep
+    //    smaller CTAs, two per SM, so the next layer's CTAs find room beside them and start early);
+    //  - mid-size batches, where a 16-CTA cluster per unit would not fit but every unit still gets
+    //    at least four SMs, for every layer kind (measured: the 8-sequence 16k-32k stack's step
+    //    640 -> 551 us and the 4-sequence 64k stack's 1296 -> 1239 us, every layer kind faster,
+    //    against 4- and 6-warp CTAs two per SM).
+    const int64_t units = int64_t(batch) * Hkv;
+    const int sms = device_sm_count();
+    const bool few_units = units * 16 <= sms && items >= 16 * kMmaWideWarps * 2;
+    const bool mid_units = units * 16 > sms && units * 4 <= sms;
+    const bool wide = DELTA_WIDE && dtype == DELTA_BF16 && (few_units || mid_units);
     if (wide) return plan_variant(dtype, D, batch, Hkv, items, kVarWide);
     // 6 warps with 2 stages each (the same shared memory and pages in flight as 4 warps x 3 stages,
     // spread over more warps) for three kinds of list:
