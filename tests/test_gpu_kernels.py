@@ -154,10 +154,12 @@ SELECT_CASES = [
     (5, 1, 64, "f32", [400], 0, 0, 0, 0),           # nothing selected
     (2, 2, 128, "bf16", [700], 1, 0, 0, 8),         # k = 1, no sink, no recency
     (8, 1, 128, "f32", [16], 4, 16, 64, 0),         # one-page context
-    # 11,875 pages with 4-warp, 64-column CTAs: more order keys than the selecting CTA's idle shared
-    # memory holds (about 11,100), so the selection keeps them in the workspace
-    (2, 8, 64, "bf16", [190000, 120000], 300, 16, 512, 32),
-    # 28,125 pages in one 8-warp cluster: the longest lists the selection accepts in shared memory
+    # 16 units (a mid-size batch: 8-warp CTAs, 64 columns, 96 KB of stages): 23,750 pages per sequence
+    # are more order keys than the selecting CTA's idle shared memory holds (about 22,300), so the
+    # selection keeps them in the workspace, one row per sequence
+    (2, 8, 64, "bf16", [380000, 240000], 300, 16, 512, 32),
+    # 28,125 pages of one sequence in one 16-CTA cluster: close to the longest list the selection
+    # accepts (32,768 pages); order keys in the workspace
     (8, 1, 64, "bf16", [450000], 300, 16, 512, 32),
     # 48 sequences x 8 KV heads = 384 units, more than one wave of CTAs: tickets across waves
     (4, 8, 128, "bf16", [100 + 61 * i for i in range(48)], 16, 16, 64, 8),
