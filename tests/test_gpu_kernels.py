@@ -93,6 +93,10 @@ FULL_CASES = [
     (2, 2, 64, "bf16", [16, 32]),
     (6, 1, 128, "bf16", [513]),
     (8, 8, 128, "bf16", [2500, 1, 64]),
+    # few units and long contexts: each unit's splits form several clusters, whose partials meet in
+    # the workspace (the last CTA of each (sequence, KV head) merges them)
+    (4, 2, 128, "bf16", [150000, 9000]),
+    (2, 1, 64, "f32", [100000]),
 ]
 
 
