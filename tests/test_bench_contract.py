@@ -112,3 +112,13 @@ def test_selection_quality_overlap_and_planted_recall():
     assert r["delta_layers_mean"] == 1.0 and 0.0 < r["served_layers_mean"] < 1.0
     ov = q["step_overlap"]
     assert ov["mean_other_steps"] == 1.0 and ov["mean_at_drift_steps"] < 1.0
+
+
+def test_planted_logit_boost_reports_the_rise_of_planted_keys():
+    import bench
+    cfg = C.QWEN7B_8K.with_(num_layers=4, delta_layers=(2,))
+    q = bench.planted_logit_boost(cfg, Case(cfg), [2])
+    # k <- 0.5 k + 3 q_hat with q_hat the unit mean of the group's queries: about 3 |q| cos / sqrt(D)
+    assert 0.8 < q["mean_rise_nats"] < 1.6
+    assert 0.9 < q["unplanted_logit_std"] < 1.1
+    assert bench.planted_logit_boost(C.TINY, Case(C.TINY), [1]) is None   # nothing planted
